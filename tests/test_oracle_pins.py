@@ -1,0 +1,353 @@
+"""Pins for the CPU oracle against facts fixed by the mathematics.
+
+Each test ties one oracle step to something other than the oracle itself: a
+library routine (torch's scaled_dot_product_attention), a closed form, an
+invariant of attention (Lemma 3.1, Lemma 3.2, Theorem 3.3 of "Sparser
+Block-Sparse Attention via Token Permutation"), brute-force enumeration on
+tiny inputs, or a hand-worked example in the style of that paper's Figure 1
+(B = 1, S = 4).
+"""
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import pbs_oracle as orc
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+def rand_qkv(seed, b=1, hq=2, hkv=1, n=64, d=16):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((b, hq, n, d))
+    k = rng.standard_normal((b, hkv, n, d))
+    v = rng.standard_normal((b, hkv, n, d))
+    return q, k, v
+
+
+def sdpa(q, k, v, mask=None, causal=False, scale=None):
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+    out = F.scaled_dot_product_attention(
+        t(q), t(k), t(v), attn_mask=None if mask is None else t(mask),
+        is_causal=causal, scale=scale, enable_gqa=True)
+    return out.numpy()
+
+
+def within_segment_perm(rng, b, h, n, segment):
+    pos = np.empty((b, h, n), dtype=np.int64)
+    for bi in range(b):
+        for hi in range(h):
+            for s0 in range(0, n, segment):
+                pos[bi, hi, s0:s0 + segment] = s0 + rng.permutation(segment)
+    return pos
+
+
+# ---------------------------------------------------------------- attention
+def test_dense_causal_matches_library():
+    q, k, v = rand_qkv(0, b=2, hq=4, hkv=2, n=48, d=8)
+    np.testing.assert_allclose(orc.dense_causal(q, k, v), sdpa(q, k, v, causal=True),
+                               rtol=0, atol=1e-12)
+
+
+def test_all_blocks_identity_is_dense_causal():
+    q, k, v = rand_qkv(1, hq=4, hkv=2, n=64, d=8)
+    nb = 8
+    idx = np.tile(np.arange(nb, dtype=np.int32), (1, 4, nb, 1))
+    cnt = np.full((1, 4, nb), nb, dtype=np.int32)
+    o = orc.attend(q, k, v, None, None, idx, cnt, 8)
+    np.testing.assert_allclose(o, sdpa(q, k, v, causal=True), atol=1e-12)
+
+
+def test_theorem_3_3_permute_attend_unpermute():
+    """All blocks kept: permuting Q, K, V inside segments, attending with the
+    carried positions and inverting the query order gives dense causal."""
+    rng = np.random.default_rng(2)
+    q, k, v = rand_qkv(2, hq=4, hkv=2, n=64, d=8)
+    block, segment = 4, 16
+    kpos = within_segment_perm(rng, 1, 2, 64, segment)
+    perm = {"kpos": kpos, "k_perm": orc.gather_rows(k, kpos),
+            "v_perm": orc.gather_rows(v, kpos)}
+    qpos = np.repeat(kpos, 2, axis=1)
+    q_perm = orc.gather_rows(q, qpos)
+    nb = 64 // block
+    idx = np.tile(np.arange(nb, dtype=np.int32), (1, 4, nb, 1))
+    cnt = np.full((1, 4, nb), nb, dtype=np.int32)
+    o_perm = orc.attend(q_perm, perm["k_perm"], perm["v_perm"], kpos, qpos, idx, cnt, block)
+    np.testing.assert_allclose(orc.unpermute(o_perm, qpos), sdpa(q, k, v, causal=True),
+                               atol=1e-12)
+
+
+def test_lemma_3_2_query_equivariance():
+    """Permuting the query rows permutes the output rows the same way."""
+    rng = np.random.default_rng(3)
+    q, k, v = rand_qkv(3, hq=2, hkv=2, n=32, d=8)
+    nb = 4
+    idx = np.tile(np.arange(nb, dtype=np.int32), (1, 2, nb, 1))
+    cnt = np.full((1, 2, nb), nb, dtype=np.int32)
+    qpos = within_segment_perm(rng, 1, 2, 32, 32)
+    o = orc.attend(q, k, v, None, None, idx, cnt, 8)
+    o_p = orc.attend(orc.gather_rows(q, qpos), k, v, None, qpos, idx, cnt, 8)
+    np.testing.assert_allclose(o_p, orc.gather_rows(o, qpos), atol=1e-12)
+
+
+def test_lemma_3_1_key_value_invariance():
+    """Reordering (key, value, position) triples inside each block leaves the
+    output unchanged for any block selection."""
+    rng = np.random.default_rng(4)
+    q, k, v = rand_qkv(4, hq=2, hkv=1, n=64, d=8)
+    block, segment = 8, 32
+    imp = rng.random((1, 1, 64))
+    perm = orc.permute(imp, k, v, segment)
+    idx, cnt, _ = orc.select_blocks(orc.block_means(q, block),
+                                    orc.block_means(perm["k_perm"], block),
+                                    segment // block, "threshold", 0.5, None, 2)
+    o1 = orc.attend(q, perm["k_perm"], perm["v_perm"], perm["kpos"], None, idx, cnt, block)
+    inner = within_segment_perm(rng, 1, 1, 64, block)
+    o2 = orc.attend(q, orc.gather_rows(perm["k_perm"], inner),
+                    orc.gather_rows(perm["v_perm"], inner),
+                    np.take_along_axis(perm["kpos"], inner, axis=2), None, idx, cnt, block)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+
+
+def test_identity_permutation_is_plain_block_sparse():
+    """kpos = identity: the output is causal attention restricted to the kept
+    blocks, i.e. the library routine with that token-level mask."""
+    q, k, v = rand_qkv(5, hq=2, hkv=1, n=64, d=8)
+    block, segment = 8, 16
+    idx, cnt, _ = orc.select_blocks(orc.block_means(q, block), orc.block_means(k, block),
+                                    segment // block, "topk_frac", 0.3, None, 2)
+    o = orc.attend(q, k, v, None, None, idx, cnt, block)
+    for g in range(2):
+        blockmask = np.zeros((8, 8), dtype=bool)
+        for i in range(8):
+            blockmask[i, idx[0, g, i, :cnt[0, g, i]]] = True
+        mask = np.kron(blockmask, np.ones((block, block), dtype=bool)) & np.tril(
+            np.ones((64, 64), dtype=bool))
+        ref = sdpa(q[:, g:g + 1], k, v, mask=mask)
+        np.testing.assert_allclose(o[:, g:g + 1], ref, atol=1e-12)
+
+
+def test_single_segment_is_dense_causal():
+    """S = N: every block is in the on-diagonal segment, so the whole path
+    (with its permutation) reproduces dense causal attention."""
+    q, k, v = rand_qkv(6, hq=4, hkv=2, n=64, d=8)
+    for mode, param in (("threshold", 0.5), ("topk_frac", 0.1)):
+        res = orc.pbs_attention(q, k, v, 8, 64, mode, param)
+        np.testing.assert_allclose(res["o"], sdpa(q, k, v, causal=True), atol=1e-12)
+        res = orc.pbs_attention(q, k, v, 8, 64, mode, param, permute_q=True)
+        np.testing.assert_allclose(res["o"], sdpa(q, k, v, causal=True), atol=1e-12)
+
+
+def test_segment_equal_block_selection_ignores_permutation():
+    """S = B: a block is a segment, so its mean key (and the lists) cannot
+    depend on the order inside it."""
+    q, k, v = rand_qkv(7, hq=2, hkv=1, n=64, d=8)
+    rng = np.random.default_rng(7)
+    imp = rng.random((1, 1, 64))
+    perm = orc.permute(imp, k, v, 8)
+    a = orc.select_blocks(orc.block_means(q, 8), orc.block_means(perm["k_perm"], 8), 1,
+                          "threshold", 0.8, None, 2)
+    b = orc.select_blocks(orc.block_means(q, 8), orc.block_means(k, 8), 1,
+                          "threshold", 0.8, None, 2)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_all_mode_after_permutation_is_dense_causal():
+    q, k, v = rand_qkv(8, hq=4, hkv=1, n=96, d=8)
+    res = orc.pbs_attention(q, k, v, 8, 32, "all", 0.0)
+    np.testing.assert_allclose(res["o"], sdpa(q, k, v, causal=True), atol=1e-12)
+    res = orc.pbs_attention(q, k, v, 8, 32, "all", 0.0, permute_q=True)
+    np.testing.assert_allclose(res["o"], sdpa(q, k, v, causal=True), atol=1e-12)
+
+
+# ---------------------------------------------------------------- scoring
+def test_score_equals_library_attention_probabilities():
+    """Attention against V = identity returns the probability matrix itself,
+    so the mean over the probe rows must equal the importance."""
+    q, k, _ = rand_qkv(9, b=2, hq=4, hkv=2, n=40, d=8)
+    block = 8
+    imp = orc.score(q, k, block)
+    n = 40
+    eye = np.eye(n)[None, None]
+    mask = np.arange(n)[None, :] <= np.arange(n - block, n)[:, None]
+    for bi in range(2):
+        for h in range(2):
+            rows = q[bi:bi + 1, 2 * h:2 * h + 2, n - block:]
+            p = sdpa(rows, k[bi:bi + 1, h:h + 1], eye, mask=mask)  # [1, 2, block, n]
+            np.testing.assert_allclose(imp[bi, h], p.reshape(-1, n).mean(0), atol=1e-14)
+
+
+def test_score_closed_forms():
+    # one probe row that sees exactly one key
+    q = np.ones((1, 1, 1, 4))
+    k = np.ones((1, 1, 1, 4))
+    assert orc.score(q, k, 1)[0, 0, 0] == 1.0
+    # identical keys: row at offset r sees r+1 keys uniformly
+    n = block = 6
+    q, _, _ = rand_qkv(10, hq=1, hkv=1, n=n, d=4)
+    k = np.ones((1, 1, n, 4))
+    want = [sum(1.0 / (r + 1) for r in range(j, n)) / n for j in range(n)]
+    np.testing.assert_allclose(orc.score(q, k, block)[0, 0], want, atol=1e-15)
+    # rows sum to one; keys after the last position carry no weight
+    q, k, _ = rand_qkv(11, hq=4, hkv=1, n=32, d=8)
+    imp = orc.score(q, k, 8)
+    assert abs(imp.sum() - 1.0) < 1e-12
+
+
+# ------------------------------------------------------------- permutation
+def test_segment_order_sorts_descending_with_stable_ties():
+    rng = np.random.default_rng(12)
+    imp = rng.random((2, 3, 48)).round(1)        # many exact ties
+    kpos = orc.segment_order(imp, 16)
+    for bi in range(2):
+        for h in range(3):
+            for s0 in range(0, 48, 16):
+                seg = kpos[bi, h, s0:s0 + 16]
+                assert sorted(seg.tolist()) == list(range(s0, s0 + 16))
+                vals = imp[bi, h, seg]
+                assert np.all(vals[:-1] >= vals[1:])
+                for p in range(15):
+                    if vals[p] == vals[p + 1]:
+                        assert seg[p] < seg[p + 1]
+
+
+def test_figure1_style_worked_example():
+    """B = 1, S = 4, N = 8, d = 1 (the setting of Figure 1), worked by hand.
+
+    All queries are 1, so the last row's logits are the keys themselves and
+    the importance is softmax(k). Keys [0.5, 2, -1, 2 | 1, 0, 3, -2]:
+    segment 0 sorts to original indices [1, 3, 0, 2] (tie 2 = 2 keeps 1
+    before 3), segment 1 to [6, 4, 5, 7]. Block scores of query block 7 are
+    the permuted keys [2, 2, .5, -1, 3, 1, 0, -2]; the own segment holds
+    (e^3 + e + 1 + e^-2) / Z = 0.5877 of the mass, so tau = 0.9 adds slot 0
+    (mass 0.7691) and slot 1 (0.9505) and stops.
+    """
+    k = np.array([0.5, 2, -1, 2, 1, 0, 3, -2]).reshape(1, 1, 8, 1)
+    q = np.ones((1, 1, 8, 1))
+    v = np.arange(8, dtype=float).reshape(1, 1, 8, 1)
+    res = orc.pbs_attention(q, k, v, 1, 4, "threshold", 0.9)
+    assert res["kpos"][0, 0].tolist() == [1, 3, 0, 2, 6, 4, 5, 7]
+    lists = [res["idx"][0, 0, i, :res["cnt"][0, 0, i]].tolist() for i in range(8)]
+    assert lists[:4] == [[0, 1, 2, 3]] * 4
+    assert lists[7] == [0, 1, 4, 5, 6, 7]
+    # row 7 attends to original keys 1, 3 (slots 0, 1) and 4..7
+    ks = [2, 2, 1, 0, 3, -2]
+    vs = [1, 3, 4, 5, 6, 7]
+    z = sum(math.exp(x) for x in ks)
+    o7 = sum(math.exp(x) * y for x, y in zip(ks, vs)) / z
+    assert abs(res["o"][0, 0, 7, 0] - o7) < 1e-12
+    # top-k with f = 0.75: k_I = floor(0.75 (I+1)) -> 3, 4, 5, 6 for I = 4..7
+    res = orc.pbs_attention(q, k, v, 1, 4, "topk_frac", 0.75)
+    lists = [res["idx"][0, 0, i, :res["cnt"][0, 0, i]].tolist() for i in range(8)]
+    assert lists[4:] == [[4, 5, 6, 7], [4, 5, 6, 7], [0, 4, 5, 6, 7], [0, 1, 4, 5, 6, 7]]
+    # segment 0 under top-k: k_I = max(1, floor(.75 (I+1))) < 4 = |own segment|
+    assert lists[:4] == [[0, 1, 2, 3]] * 4
+
+
+# --------------------------------------------------------------- selection
+def _rows_of(q, k, block, segment, seed):
+    idx = orc.block_means(q, block)
+    kb = orc.block_means(k, block)
+    return idx, kb
+
+
+def test_block_score_is_mean_of_token_logits():
+    """sigma * mean(Q_I) . mean(K_J) = mean over the B x B token logits."""
+    q, k, _ = rand_qkv(13, hq=1, hkv=1, n=32, d=8)
+    B = 8
+    qb, kb = orc.block_means(q, B), orc.block_means(k, B)
+    sigma = orc.resolve_scale(None, 8)
+    tok = sigma * q[0, 0] @ k[0, 0].T
+    for i in range(4):
+        for j in range(4):
+            want = tok[i * B:(i + 1) * B, j * B:(j + 1) * B].mean()
+            assert abs(sigma * qb[0, 0, i] @ kb[0, 0, j] - want) < 1e-13
+
+
+@pytest.mark.parametrize("tau", [0.3, 0.6, 0.9, 0.97])
+def test_threshold_selection_brute_force(tau):
+    """Among all subsets T of earlier-segment blocks whose mass with the own
+    segment reaches tau, the kept set is the one of least size and, at that
+    size, of largest mass."""
+    rng = np.random.default_rng(int(tau * 100))
+    spb, nseg = 2, 4
+    nb = spb * nseg
+    for trial in range(6):
+        a_all = rng.standard_normal(nb) * 1.5
+        for i in range(nb):
+            seg = i // spb
+            adm = (seg + 1) * spb
+            a = a_all[:adm]
+            kept, _ = orc.select_row(a, i, spb, "threshold", tau)
+            pi = np.exp(a - a.max())
+            pi /= pi.sum()
+            forced = set(range(seg * spb, adm))
+            earlier = range(seg * spb)
+            best = None
+            for r in range(len(earlier) + 1):
+                for t in itertools.combinations(earlier, r):
+                    m = pi[list(forced | set(t))].sum()
+                    if m >= np.float32(tau) and (best is None or m > best[1]):
+                        best = (set(t), m)
+                if best is not None:
+                    break
+            if best is None:          # tau unreachable: everything admissible
+                best = (set(earlier), 1.0)
+            assert set(kept.tolist()) == forced | best[0]
+
+
+@pytest.mark.parametrize("frac", [0.1, 0.25, 0.5, 0.9])
+def test_topk_selection_brute_force(frac):
+    rng = np.random.default_rng(int(frac * 100))
+    spb, nseg = 2, 4
+    nb = spb * nseg
+    for trial in range(4):
+        a_all = rng.standard_normal(nb)
+        for i in range(nb):
+            seg = i // spb
+            a = a_all[:(seg + 1) * spb]
+            kept, _ = orc.select_row(a, i, spb, "topk_frac", frac)
+            k_i = max(1, math.floor(float(np.float32(frac)) * (i + 1)))
+            extra = min(seg * spb, max(0, k_i - spb))
+            best = max(itertools.combinations(range(seg * spb), extra),
+                       key=lambda t: sum(a[list(t)]))
+            assert set(kept.tolist()) == set(range(seg * spb, (seg + 1) * spb)) | set(best)
+
+
+def test_select_lists_are_ascending_and_admissible():
+    q, k, v = rand_qkv(14, hq=4, hkv=2, n=128, d=8)
+    res = orc.pbs_attention(q, k, v, 8, 32, "threshold", 0.9)
+    idx, cnt = res["idx"], res["cnt"]
+    for g in range(4):
+        for i in range(16):
+            lst = idx[0, g, i, :cnt[0, g, i]]
+            assert np.all(np.diff(lst) > 0)
+            seg = i // 4
+            assert set(range(seg * 4, seg * 4 + 4)) <= set(lst.tolist())
+            assert lst.max() < (seg + 1) * 4
+            assert np.all(idx[0, g, i, cnt[0, g, i]:] == -1)
+
+
+def test_bf16_block_sums_are_exact():
+    """fp64 block sums of bf16 inputs are exact for the synthetic workloads,
+    so any summation order gives the same bits."""
+    from long_context_sparse_segment_b200.workloads import WORKLOADS, make_inputs
+    q, k, v, _ = make_inputs(WORKLOADS["tiny"])
+    x = k.double().numpy()[0, 0]
+    B = 64
+    for j in range(0, 1024, B):
+        for t in range(0, 64, 7):
+            exact = sum(Fraction(float(val)) for val in x[j:j + B, t])
+            assert Fraction(float(x[j:j + B, t].sum())) == exact
+
+
+def test_unpermute_inverts_gather():
+    rng = np.random.default_rng(15)
+    x = rng.standard_normal((2, 3, 32, 4))
+    pos = within_segment_perm(rng, 2, 3, 32, 8)
+    np.testing.assert_array_equal(orc.unpermute(orc.gather_rows(x, pos), pos), x)
