@@ -148,16 +148,17 @@ def block_means(x, block):
 def select_row(a, i_blk, spb, mode, param):
     """Kept key blocks of query block ``i_blk`` (ascending) and a margin.
 
-    a: block scores of the admissible key blocks 0 .. (seg(I)+1)*spb - 1.
+    a: block scores of the admissible key blocks 0 .. (seg(I)+1)*spb - 1,
+    cut at the last block (a shorter last segment has fewer blocks).
     The margin is the smallest gap that decides the result: for THRESHOLD
     the distance of the kept mass to tau on either side of the cut and the
     score gap at the cut; for TOPK_FRAC the score gap at the cut. It is
     +inf where nothing is decided.
     """
     seg = i_blk // spb
-    forced = np.arange(seg * spb, (seg + 1) * spb)
+    forced = np.arange(seg * spb, len(a))
     if mode == "all":
-        return np.arange((seg + 1) * spb), math.inf
+        return np.arange(len(a)), math.inf
     if mode == "dense_causal":
         return np.arange(i_blk + 1), math.inf
     n_earlier = seg * spb
@@ -184,7 +185,7 @@ def select_row(a, i_blk, spb, mode, param):
     elif mode == "topk_frac":
         frac = float(np.float64(np.float32(param)))
         k_i = max(1, math.floor(frac * (i_blk + 1)))
-        taken = min(n_earlier, max(0, k_i - spb))
+        taken = min(n_earlier, max(0, k_i - len(forced)))
         if 0 < taken < n_earlier:
             margin = a[order[taken - 1]] - a[order[taken]]
     else:
@@ -211,7 +212,7 @@ def select_blocks(q_pooled, k_pooled, spb, mode, param, scale, group):
             kb = k_pooled[bi, g // group]
             scores = sigma * (q_pooled[bi, g] @ kb.T)          # [nb, nb]
             for i in range(nb):
-                adm = ((i // spb) + 1) * spb
+                adm = min(nb, ((i // spb) + 1) * spb)
                 kept, mg = select_row(scores[i, :adm], i, spb, mode, param)
                 idx[bi, g, i, :len(kept)] = kept
                 cnt[bi, g, i] = len(kept)

@@ -157,11 +157,12 @@ def test_segment_equal_block_selection_ignores_permutation():
     np.testing.assert_array_equal(a[1], b[1])
 
 
-def test_all_mode_after_permutation_is_dense_causal():
+@pytest.mark.parametrize("segment", [32, 64])        # 64: shorter last segment
+def test_all_mode_after_permutation_is_dense_causal(segment):
     q, k, v = rand_qkv(8, hq=4, hkv=1, n=96, d=8)
-    res = orc.pbs_attention(q, k, v, 8, 32, "all", 0.0)
+    res = orc.pbs_attention(q, k, v, 8, segment, "all", 0.0)
     np.testing.assert_allclose(res["o"], sdpa(q, k, v, causal=True), atol=1e-12)
-    res = orc.pbs_attention(q, k, v, 8, 32, "all", 0.0, permute_q=True)
+    res = orc.pbs_attention(q, k, v, 8, segment, "all", 0.0, permute_q=True)
     np.testing.assert_allclose(res["o"], sdpa(q, k, v, causal=True), atol=1e-12)
 
 
@@ -317,6 +318,14 @@ def test_topk_selection_brute_force(frac):
             best = max(itertools.combinations(range(seg * spb), extra),
                        key=lambda t: sum(a[list(t)]))
             assert set(kept.tolist()) == set(range(seg * spb, (seg + 1) * spb)) | set(best)
+
+
+def test_shorter_last_segment_forces_its_own_blocks():
+    q, k, v = rand_qkv(16, hq=2, hkv=1, n=96, d=8)
+    res = orc.pbs_attention(q, k, v, 8, 64, "topk_frac", 0.05)
+    for i in range(8, 12):          # query blocks of the 4-block last segment
+        assert res["idx"][0, 0, i, :res["cnt"][0, 0, i]].tolist() == [8, 9, 10, 11]
+    assert res["kpos"][0, 0, 64:].min() == 64
 
 
 def test_select_lists_are_ascending_and_admissible():
