@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the permuted block-sparse attention (PBS-Attn) prefill path.
+
+One step = the whole path over one synthetic input (every layer of it):
+importance scoring, segment-local permutation, block selection and the
+block-sparse forward (the inverse permutation is a no-op in the default
+natural-query mode). Inputs are resident in HBM before timing and larger
+than L2. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+  python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Under torchrun every rank runs its own replica of the workload (the units of
+the path are independent per batch and head, so there is no collective on the
+data path): weak scaling, value = all ranks' work / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import long_context_sparse_segment_b200 as pbs  # noqa: E402
+from long_context_sparse_segment_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "PBS-Attn prefill ms and effective TFLOP/s (% BF16 peak) at N=32K–128K vs dense"
+UNIT = "TFLOP/s"
+LAUNCHES_PER_LAYER = 8  # score 3, permute 2, select 2, forward 1
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="llama128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def block_flops(w, total_blocks):
+    return 4.0 * w.block * w.block * w.d * total_blocks
+
+
+# ------------------------------------------------------------------ clocks
+REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while timing."""
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", ident, "--query-gpu=clocks.sm,clocks.max.sm,power.draw,"
+                 "clocks_event_reasons.active", "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 4:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                    mask = int(parts[3], 16)
+                except ValueError:
+                    continue
+                for bit, name in REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- GPU arm
+class Layer:
+    def __init__(self, w, dev, layer, seed_offset):
+        self.w = w
+        self.q, self.k, self.v, _ = make_inputs(w, dev, layer=layer, seed=w.seed + layer + seed_offset)
+        self.out = None
+
+
+def run_layer(layer, ev=None):
+    """The five steps on one layer; returns (o, blk_cnt). ev: dict of event
+    pairs recorded around score / permute / select / forward."""
+    w = layer.w
+    B, S = w.block, w.segment
+
+    def mark(name, i):
+        if ev is not None:
+            ev[name][i].record()
+
+    mark("score", 0)
+    imp = pbs.score(layer.q, layer.k, B, S)
+    mark("score", 1)
+    mark("permute", 0)
+    perm = pbs.permute(imp, layer.k, layer.v, B, S, hq=w.hq)
+    mark("permute", 1)
+    mark("select", 0)
+    idx, cnt, _ = pbs.select_blocks(layer.q, perm["k_perm"], perm["kbar_sum"], B, S, w.mode,
+                                    w.param)
+    mark("select", 1)
+    mark("attn", 0)
+    o = pbs.attn_fwd(layer.q, perm["k_perm"], perm["v_perm"], perm["kpos"], None, idx, cnt, B,
+                     S, out=layer.out)
+    mark("attn", 1)
+    layer.out = o
+    return o, cnt
+
+
+def time_dense(layer, reps=3):
+    """Plain causal attention (identity order, blocks J <= I) on the same
+    forward kernel, for the speedup."""
+    w = layer.w
+    idx, cnt, _ = pbs.select_blocks(layer.q, layer.k, None, w.block, w.segment, "dense_causal")
+    for _ in range(2):
+        pbs.attn_fwd(layer.q, layer.k, layer.v, None, None, idx, cnt, w.block, w.segment,
+                     out=layer.out)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        pbs.attn_fwd(layer.q, layer.k, layer.v, None, None, idx, cnt, w.block, w.segment,
+                     out=layer.out)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps, float(cnt.sum().item())
+
+
+def e2e_run(w, layers, steps):
+    """The same metric through the public call with host buffers: every step
+    copies the inputs from pinned host memory, runs the path and reads the
+    output back."""
+    host = []
+    for L in layers:
+        host.append(tuple(t.cpu().pin_memory() for t in (L.q, L.k, L.v)))
+    o_host = torch.empty(layers[0].q.shape, dtype=torch.bfloat16).pin_memory()
+    dq = torch.empty_like(layers[0].q)
+    dk = torch.empty_like(layers[0].k)
+    dv = torch.empty_like(layers[0].v)
+    h2d = sum(t.numel() * t.element_size() for t in host[0]) * len(layers)
+    d2h = o_host.numel() * o_host.element_size() * len(layers)
+
+    def one():
+        for hq_, hk_, hv_ in host:
+            dq.copy_(hq_, non_blocking=True)
+            dk.copy_(hk_, non_blocking=True)
+            dv.copy_(hv_, non_blocking=True)
+            o = pbs.pbs_attention(dq, dk, dv, w.block, w.segment, w.mode, w.param)
+            o_host.copy_(o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def gpu_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w = WORKLOADS[args.config]
+    layers = [Layer(w, dev, l, seed_offset=1000 * rank) for l in range(w.layers)]
+    torch.cuda.synchronize()
+
+    # warm-up (also fixes the kept-block counts of this input)
+    for _ in range(max(3, args.warmup)):
+        total_blocks = 0.0
+        for L in layers:
+            _, cnt = run_layer(L)
+            total_blocks += float(cnt.sum().item())
+    flops_per_step = block_flops(w, total_blocks)
+
+    names = ("score", "permute", "select", "attn")
+    evs = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for n in names} for _ in range(args.steps * len(layers))]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
+    start.record()
+    i = 0
+    for _ in range(args.steps):
+        for L in layers:
+            run_layer(L, evs[i])
+            i += 1
+    stop.record()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    if dist:
+        dist.barrier()
+    ms = start.elapsed_time(stop) / args.steps
+    per = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) / args.steps for n in names}
+    attn_launch_ms = per["attn"] / len(layers)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    value = flops_per_step * world / (ms * 1e-3) / 1e12
+    pk, pk_kind = peaks()
+    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    attn_tflops = flops_per_step / len(layers) / (attn_launch_ms * 1e-3) / 1e12
+
+    dense_ms, dense_blocks = time_dense(layers[0])
+    e2e_ms, h2d, d2h = e2e_run(w, layers, max(1, args.e2e_steps))
+    e2e_value = flops_per_step * world / (e2e_ms * 1e-3) / 1e12
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        e2e_value = flops_per_step * world / (e2e_ms * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 with planted salient keys)",
+        "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "n": w.n,
+                   "d": w.d, "block": w.block, "segment": w.segment, "layers": w.layers,
+                   "selection": f"{w.mode} {w.param}", "l2": "inputs larger than L2",
+                   "parallelism": f"replicas x{world}"},
+        "density": round(total_blocks / max(1.0, dense_blocks * len(layers)), 4),
+        "breakdown_ms": {n: round(v, 4) for n, v in per.items()},
+        "dense_attn_ms": round(dense_ms * len(layers), 4),
+        "speedup_vs_dense": {"attn": round(dense_ms / attn_launch_ms, 3),
+                             "path": round(dense_ms * len(layers) / ms, 3)},
+        "clocks": clock_info,
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "ms_per_step": round(e2e_ms, 3),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": LAUNCHES_PER_LAYER * len(layers) * args.steps,
+        "roofline": {"kernel": "pbs_attn_fwd", "bound": "tensor",
+                     "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / peak, 4), "peak_kind":
+                     f"{pk_kind} bf16 dense, sustained", "traffic": traffic_for(w)},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, layers[0], total_blocks / len(layers))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def traffic_for(w):
+    """DRAM bytes per forward launch from the committed ncu summary, if one
+    exists for this workload."""
+    path = os.path.join(ROOT, "profiles", "attn_fwd_dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 2 and parts[0] == w.name:
+                try:
+                    return float(parts[1])
+                except ValueError:
+                    return None
+    return None
+
+
+# ---------------------------------------------------------- the CPU oracle
+def oracle_sample(w, q, k, v, blocks_total_hint=None, attn_blocks=8):
+    """Time the oracle on one KV group of the workload and scale it up.
+
+    q: [1, G, n, d], k, v: [1, 1, n, d] bf16 CPU tensors of one KV group.
+    Score, permutation and selection of the group are timed in full and
+    scaled by the number of (batch, KV head) groups; the forward is timed on
+    `attn_blocks` query blocks of the first head and scaled by kept blocks.
+    Returns (seconds for the whole workload, total kept blocks, sample text).
+    """
+    import numpy as np
+
+    from oracle import pbs_oracle as orc
+    B, S = w.block, w.segment
+    groups = w.batch * w.hkv * w.layers
+    q64, k64, v64 = (t.double().numpy() for t in (q, k, v))
+    t0 = time.perf_counter()
+    imp = orc.score(q64, k64, B)
+    t1 = time.perf_counter()
+    perm = orc.permute(imp, k64, v64, S)
+    t2 = time.perf_counter()
+    idx, cnt, _ = orc.select_blocks(orc.block_means(q64, B), orc.block_means(perm["k_perm"], B),
+                                    S // B, w.mode, w.param, None, w.group)
+    t3 = time.perf_counter()
+    nb = w.nb
+    picks = sorted({int(round(x)) for x in np.linspace(0, nb - 1, attn_blocks)})
+    blocks = [(0, 0, i) for i in picks]
+    orc.attend_blocks(q64, perm["k_perm"], perm["v_perm"], perm["kpos"], None, idx, cnt, B,
+                      blocks)
+    t4 = time.perf_counter()
+    sampled = float(sum(cnt[0, 0, i] for i in picks))
+    group_blocks = float(cnt.sum())
+    total_blocks = group_blocks * groups
+    per_block = (t4 - t3) / sampled
+    seconds = (t3 - t0) * groups + per_block * total_blocks
+    text = (f"KV group 0 at full n={w.n}: score {t1 - t0:.2f}s, permute {t2 - t1:.2f}s, "
+            f"select {t3 - t2:.2f}s timed in full and scaled x{groups} groups; forward on "
+            f"{len(picks)} query blocks of head 0 ({int(sampled)} kept blocks, {t4 - t3:.2f}s) "
+            f"scaled to {int(total_blocks)} kept blocks")
+    return seconds, total_blocks, text
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, layer, blocks_per_layer):
+    G = w.group
+    q = layer.q[:1, :G].cpu()
+    k = layer.k[:1, :1].cpu()
+    v = layer.v[:1, :1].cpu()
+    seconds, total_blocks, text = oracle_sample(w, q, k, v)
+    value = block_flops(w, total_blocks) / seconds / 1e12
+    return {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": text, "ms_per_step_extrapolated": round(seconds * 1e3, 1)}
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.config]
+    # one KV group of the workload, drawn on the host with the same recipe
+    wg = w.with_(batch=1, hq=w.group, hkv=1, layers=1)
+    q, k, v, _ = make_inputs(wg)
+    times, text, blocks = [], "", 0.0
+    for i in range(args.warmup + args.steps):
+        sec, blocks, text = oracle_sample(w, q, k, v)
+        if i >= args.warmup:
+            times.append(sec)
+    sec = statistics.mean(times)
+    value = block_flops(w, blocks) / sec / 1e12
+    cores = blas_threads()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": int(os.environ.get(
+            "WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "n": w.n,
+                   "d": w.d, "block": w.block, "segment": w.segment, "layers": w.layers,
+                   "selection": f"{w.mode} {w.param}"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": text},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

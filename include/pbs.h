@@ -1,0 +1,223 @@
+/*
+ * pbs.h - C ABI of libpbs, the sm_100a (B200) implementation of the prefill
+ * path of Permuted Block-Sparse Attention (PBS-Attn).
+ *
+ * Method: "Sparser Block-Sparse Attention via Token Permutation"
+ * (arXiv 2510.21270). The five calls below are its five steps:
+ *
+ *   pbs_score          key importance from the last query block
+ *   pbs_permute        segment-local key order, K/V (and Q) gathered by it
+ *   pbs_select_blocks  key blocks kept per query block, from pooled scores
+ *   pbs_attn_fwd       causal block-sparse attention on the permuted keys
+ *   pbs_unpermute      inverse permutation of the output rows
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Tensors are dense, row-major, head dim innermost, in DEVICE memory:
+ *     Q, O        [batch, hq,  n, d]  bf16
+ *     K, V, K', V'[batch, hkv, n, d]  bf16
+ *   Base pointers must be 16-byte aligned.
+ * - Query head g reads KV head g / (hq / hkv) (grouped-query attention).
+ * - Supported: d in {64, 128}, block (B) in {64, 128}, segment (S) a
+ *   multiple of B, n a multiple of B (the last segment may be shorter than
+ *   S when n is not a multiple of S), hq a multiple of hkv. n == 0 or
+ *   batch == 0 is a valid empty call that launches nothing.
+ * - scale <= 0 selects the softmax scale sigma = 1/sqrt(d).
+ * - The caller owns every buffer, the workspace included; the library never
+ *   allocates, frees or keeps a pointer after a call returns.
+ * - Calls are asynchronous on the given stream (a cudaStream_t; NULL is the
+ *   legacy default stream). Argument errors are returned synchronously and
+ *   launch nothing. Errors found by a kernel (a wait that ran out, an index
+ *   out of range) are recorded in a per-device error word that
+ *   pbs_get_device_status reads. Nothing throws across this ABI.
+ */
+#ifndef PBS_H
+#define PBS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *pbs_stream_t; /* same type as cudaStream_t */
+
+typedef struct {
+  int batch;   /* b */
+  int hq;      /* query heads */
+  int hkv;     /* key/value heads, divides hq */
+  int n;       /* sequence length N */
+  int d;       /* head dimension: 64 or 128 */
+  int block;   /* block size B of the block-sparse attention: 64 or 128 */
+  int segment; /* permutation segment size S: a multiple of B */
+} pbs_shape;
+
+typedef enum {
+  PBS_OK = 0,
+  PBS_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or mode */
+  PBS_ERR_UNSUPPORTED = 2,   /* d or B outside the compiled kernels */
+  PBS_ERR_CUDA = 3,          /* a CUDA runtime call failed */
+  PBS_ERR_TIMEOUT = 4,       /* a kernel's bounded wait ran out */
+  PBS_ERR_DEVICE_ASSERT = 5, /* a kernel found an index out of range */
+  PBS_ERR_WORKSPACE = 6      /* workspace smaller than pbs_workspace_bytes */
+} pbs_status;
+
+typedef enum {
+  PBS_SEL_THRESHOLD = 0,   /* keep blocks until the kept softmax mass >= tau */
+  PBS_SEL_TOPK_FRAC = 1,   /* keep max(1, floor(f * (I + 1))) blocks */
+  PBS_SEL_ALL = 2,         /* every admissible block */
+  PBS_SEL_DENSE_CAUSAL = 3 /* blocks J <= I: plain causal attention */
+} pbs_sel_mode;
+
+typedef enum {
+  PBS_OP_SCORE = 0,
+  PBS_OP_PERMUTE = 1,
+  PBS_OP_SELECT = 2,
+  PBS_OP_ATTN = 3,
+  PBS_OP_UNPERMUTE = 4
+} pbs_op;
+
+/* Bytes of device workspace the call `op` needs for shape `s` (0 if none). */
+size_t pbs_workspace_bytes(pbs_shape s, int op);
+
+/*
+ * pbs_score - global key importance from the last query block.
+ * Source: gist.science summary of the paper, "Methodik" 3 ("Proxy-
+ * Bewertung"): importance is estimated from the last block of queries by
+ * mean pooling their attention scores.
+ *
+ * For each (batch, KV head h) the probe rows are the last B query rows of
+ * each of the G = hq/hkv query heads of h's group (G*B rows, positions
+ * n-B .. n-1). Each probe row r attends causally over all n keys with
+ * logits sigma * q_r . k_j; imp[b, h, j] is the mean over the G*B rows of
+ * the softmax probability of key j. Each imp row sums to 1.
+ *
+ *   q   [batch, hq, n, d] bf16 (only the last B rows of each head are read)
+ *   k   [batch, hkv, n, d] bf16
+ *   imp [batch, hkv, n] fp32, written
+ *   ws  device workspace of at least pbs_workspace_bytes(s, PBS_OP_SCORE)
+ */
+pbs_status pbs_score(const void *q, const void *k, float *imp, pbs_shape s,
+                     float scale, void *ws, size_t ws_bytes, pbs_stream_t st);
+
+/*
+ * pbs_permute - segment-local key permutation and gather.
+ * Source: gist.science summary, "Methodik" 2 (segmented permutation: only
+ * inside contiguous segments of S tokens, segment order kept) and 3
+ * ("Sortierung": keys sorted by descending global importance inside each
+ * segment); sciencestack.ai Lemma 3.1 (K and V permuted together).
+ *
+ * kpos[b, h, p] = the original index of the key placed at slot p: inside
+ * each segment keys are ordered by imp descending, equal values keeping the
+ * lower original index first. k_perm[b,h,p] = k[b,h,kpos[p]], likewise v.
+ * kbar_sum (optional) receives the fp64 sum of the B rows of each permuted
+ * key block: [batch, hkv, n/B, d]. With q non-NULL (permuted-query mode)
+ * q_perm[b, g, p] = q[b, g, kpos[b, g/G, p]] for every query head g.
+ *
+ *   imp         [batch, hkv, n] fp32 (no NaN)
+ *   k, v        [batch, hkv, n, d] bf16
+ *   q, q_perm   [batch, hq, n, d] bf16, both NULL or both non-NULL
+ *   k_perm, v_perm  [batch, hkv, n, d] bf16, written
+ *   kpos        [batch, hkv, n] int32, written
+ *   kbar_sum    [batch, hkv, n/B, d] fp64, written if non-NULL
+ */
+pbs_status pbs_permute(const float *imp, const void *k, const void *v,
+                       const void *q, void *k_perm, void *v_perm, void *q_perm,
+                       int32_t *kpos, double *kbar_sum, pbs_shape s,
+                       pbs_stream_t st);
+
+/*
+ * pbs_select_blocks - key blocks to compute for every query block.
+ * Source: gist.science summary, "Methodik" 4 ("Block-Auswahl": block
+ * importance by mean pooling over the permuted keys); sciencestack.ai
+ * Figure 1 caption (blocks of the on-diagonal segment are always computed);
+ * skillmd.com "Implementation Steps" (active blocks as a fraction of the
+ * block count, at least one).
+ *
+ * In fp64: qbar = mean of the B rows of query block I of head g, kbar = mean
+ * of permuted key block J of KV head g/G, a_IJ = sigma * qbar . kbar for the
+ * admissible J (segment(J) <= segment(I)), pi = softmax of a over them.
+ * The blocks of I's own segment are always kept. Then
+ *   THRESHOLD (param = tau in (0, 1]): earlier-segment blocks are added in
+ *     descending a (ties: lower J) while the kept pi mass is < tau;
+ *   TOPK_FRAC (param = f in (0, 1]): k = max(1, floor(f * (I + 1))) and the
+ *     best max(0, k - own) earlier-segment blocks are added;
+ *   ALL: every admissible block; DENSE_CAUSAL: J = 0 .. I.
+ *
+ *   q_or_qperm  [batch, hq, n, d] bf16: Q, or Q' in permuted-query mode
+ *   k_perm      [batch, hkv, n, d] bf16; read only when kbar_sum is NULL
+ *   kbar_sum    [batch, hkv, n/B, d] fp64 from pbs_permute, or NULL
+ *   blk_idx     [batch, hq, n/B, n/B] int32, written: row (b, g, I) holds
+ *               blk_cnt[b, g, I] ascending block indices, the rest untouched
+ *   blk_cnt     [batch, hq, n/B] int32, written
+ *   blk_mask    [batch, hq, n/B, n/B] uint8 (1 = kept), written if non-NULL
+ *   ws          device workspace of pbs_workspace_bytes(s, PBS_OP_SELECT)
+ */
+pbs_status pbs_select_blocks(const void *q_or_qperm, const void *k_perm,
+                             const double *kbar_sum, pbs_shape s, int mode,
+                             float param, float scale, int32_t *blk_idx,
+                             int32_t *blk_cnt, uint8_t *blk_mask, void *ws,
+                             size_t ws_bytes, pbs_stream_t st);
+
+/*
+ * pbs_attn_fwd - causal block-sparse attention over the permuted keys.
+ * Source: sciencestack.ai Figure 1 caption (causality kept across segments,
+ * on-diagonal segments computed) and Lemma 3.1 / 3.2; gist.science
+ * summary, "Methodik" 4 (permuted FlashAttention kernel).
+ *
+ * For query row i of head g in query block I, the visible keys are the
+ * slots p of the kept blocks of (g, I) whose original position kpos[p] is
+ * <= the query's original position (qpos[i], or i when qpos is NULL). The
+ * output row is the softmax(sigma * q_i . k'_p)-weighted sum of v'_p, in
+ * the order of the given queries (permuted order when qpos is non-NULL).
+ *
+ *   q_or_qperm      [batch, hq, n, d] bf16
+ *   k_perm, v_perm  [batch, hkv, n, d] bf16
+ *   kpos            [batch, hkv, n] int32, or NULL for the identity
+ *   qpos            [batch, hkv, n] int32 (the order of each KV group's
+ *                   queries, as from pbs_permute), or NULL = natural order
+ *   blk_idx, blk_cnt  as written by pbs_select_blocks; every list must
+ *                   hold the query block's own segment so that every row
+ *                   sees at least one key
+ *   out             [batch, hq, n, d] bf16, written
+ *   lse             [batch, hq, n] fp32 natural-log sum of exp, or NULL
+ */
+pbs_status pbs_attn_fwd(const void *q_or_qperm, const void *k_perm,
+                        const void *v_perm, const int32_t *kpos,
+                        const int32_t *qpos, const int32_t *blk_idx,
+                        const int32_t *blk_cnt, void *out, float *lse,
+                        pbs_shape s, float scale, pbs_stream_t st);
+
+/*
+ * pbs_unpermute - inverse permutation of the output rows.
+ * Source: skillmd.com "Implementation Steps" (output[argsort(perm)]);
+ * sciencestack.ai Theorem 3.3 (permute, attend, un-permute recovers the
+ * original result).
+ *
+ * out[b, g, qpos[b, g/G, p]] = out_perm[b, g, p]. With qpos NULL (natural
+ * query order) this is a copy, or nothing when out == out_perm.
+ *
+ *   out_perm, out  [batch, hq, n, d] bf16 (must not overlap unless equal)
+ *   qpos           [batch, hkv, n] int32 or NULL
+ */
+pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out,
+                         pbs_shape s, pbs_stream_t st);
+
+/*
+ * Synchronises `st`, returns in *code the current device's error word
+ * (a pbs_status; PBS_OK when no kernel reported a problem) and clears it.
+ */
+pbs_status pbs_get_device_status(pbs_stream_t st, int *code);
+
+/* Static, human-readable name of a status. */
+const char *pbs_status_string(int status);
+
+/* Library version string. */
+const char *pbs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PBS_H */

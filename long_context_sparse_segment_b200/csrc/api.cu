@@ -1,0 +1,231 @@
+// The C ABI of libpbs: argument checks, workspace layout, the device error
+// word, and the launches of the five steps. Declared in include/pbs.h.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/pbs.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace pbs {
+
+// One error word per device: kernels record the first problem they meet.
+__device__ int g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int *g_err_ptr[kMaxDevices];
+std::once_flag g_err_once[kMaxDevices];
+
+int *error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::call_once(g_err_once[dev], [dev] {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) g_err_ptr[dev] = (int *)p;
+  });
+  return g_err_ptr[dev];
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+pbs_status check_shape(const pbs_shape &s, Dims *dm) {
+  if (s.batch < 0 || s.hq < 1 || s.hkv < 1 || s.n < 0 || s.block < 1 || s.segment < 1)
+    return PBS_ERR_INVALID_ARG;
+  if (s.hq % s.hkv != 0) return PBS_ERR_INVALID_ARG;
+  if (s.d != 64 && s.d != 128) return PBS_ERR_UNSUPPORTED;
+  if (s.block != 64 && s.block != 128) return PBS_ERR_UNSUPPORTED;
+  if (s.segment % s.block != 0 || s.n % s.block != 0) return PBS_ERR_INVALID_ARG;
+  if (s.segment > 8192) return PBS_ERR_UNSUPPORTED;
+  dm->b = s.batch;
+  dm->hq = s.hq;
+  dm->hkv = s.hkv;
+  dm->n = s.n;
+  dm->d = s.d;
+  dm->B = s.block;
+  dm->S = s.segment;
+  dm->G = s.hq / s.hkv;
+  dm->nb = s.n / s.block;
+  dm->spb = s.segment / s.block;
+  dm->nseg = (s.n + s.segment - 1) / s.segment;
+  return PBS_OK;
+}
+
+bool empty(const Dims &dm) { return dm.b == 0 || dm.n == 0; }
+
+pbs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PBS_OK : PBS_ERR_CUDA; }
+
+double resolve_sigma(float scale, int d) {
+  return scale > 0.f ? (double)scale : 1.0 / sqrt((double)d);
+}
+
+}  // namespace
+}  // namespace pbs
+
+using namespace pbs;
+
+extern "C" {
+
+size_t pbs_workspace_bytes(pbs_shape s, int op) {
+  Dims dm;
+  if (check_shape(s, &dm) != PBS_OK || empty(dm)) return 0;
+  switch (op) {
+    case PBS_OP_SCORE:
+      return score_ws_bytes(dm);
+    case PBS_OP_SELECT:
+      return select_ws_bytes(dm, true);
+    default:
+      return 0;
+  }
+}
+
+pbs_status pbs_score(const void *q, const void *k, float *imp, pbs_shape s, float scale,
+                     void *ws, size_t ws_bytes, pbs_stream_t st) {
+  Dims dm;
+  pbs_status r = check_shape(s, &dm);
+  if (r != PBS_OK) return r;
+  if (empty(dm)) return PBS_OK;
+  if (!q || !k || !imp || !ws || !aligned16(q) || !aligned16(k) || !aligned16(ws) ||
+      ((uintptr_t)imp & 3u))
+    return PBS_ERR_INVALID_ARG;
+  if (!score_supported(dm)) return PBS_ERR_UNSUPPORTED;
+  if (ws_bytes < score_ws_bytes(dm)) return PBS_ERR_WORKSPACE;
+  int *err = error_word();
+  const float sigma = (float)resolve_sigma(scale, dm.d);
+  return cuda_status(launch_score(dm, q, k, imp, sigma, ws, err, (cudaStream_t)st));
+}
+
+pbs_status pbs_permute(const float *imp, const void *k, const void *v, const void *q,
+                       void *k_perm, void *v_perm, void *q_perm, int32_t *kpos,
+                       double *kbar_sum, pbs_shape s, pbs_stream_t st) {
+  Dims dm;
+  pbs_status r = check_shape(s, &dm);
+  if (r != PBS_OK) return r;
+  if (empty(dm)) return PBS_OK;
+  if (!imp || !k || !v || !k_perm || !v_perm || !kpos) return PBS_ERR_INVALID_ARG;
+  if ((q == nullptr) != (q_perm == nullptr)) return PBS_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_perm) || !aligned16(v_perm) ||
+      !aligned16(kpos) || (q && (!aligned16(q) || !aligned16(q_perm))) ||
+      (kbar_sum && !aligned16(kbar_sum)) || ((uintptr_t)imp & 3u))
+    return PBS_ERR_INVALID_ARG;
+  if (k == k_perm || v == v_perm || (q && q == q_perm)) return PBS_ERR_INVALID_ARG;
+  int *err = error_word();
+  cudaStream_t cs = (cudaStream_t)st;
+  cudaError_t e = launch_segsort(dm, imp, kpos, err, cs);
+  if (e != cudaSuccess) return PBS_ERR_CUDA;
+  return cuda_status(launch_gather(dm, kpos, k, v, q, k_perm, v_perm, q_perm, kbar_sum, err, cs));
+}
+
+pbs_status pbs_select_blocks(const void *q_or_qperm, const void *k_perm, const double *kbar_sum,
+                             pbs_shape s, int mode, float param, float scale, int32_t *blk_idx,
+                             int32_t *blk_cnt, uint8_t *blk_mask, void *ws, size_t ws_bytes,
+                             pbs_stream_t st) {
+  Dims dm;
+  pbs_status r = check_shape(s, &dm);
+  if (r != PBS_OK) return r;
+  if (mode < PBS_SEL_THRESHOLD || mode > PBS_SEL_DENSE_CAUSAL) return PBS_ERR_INVALID_ARG;
+  if ((mode == PBS_SEL_THRESHOLD || mode == PBS_SEL_TOPK_FRAC) &&
+      !(param > 0.f && param <= 1.f))
+    return PBS_ERR_INVALID_ARG;
+  if (empty(dm)) return PBS_OK;
+  if (!blk_idx || !blk_cnt || ((uintptr_t)blk_idx & 3u) || ((uintptr_t)blk_cnt & 3u))
+    return PBS_ERR_INVALID_ARG;
+  const bool scored = mode == PBS_SEL_THRESHOLD || mode == PBS_SEL_TOPK_FRAC;
+  if (scored) {
+    if (!q_or_qperm || !aligned16(q_or_qperm)) return PBS_ERR_INVALID_ARG;
+    if (!kbar_sum && (!k_perm || !aligned16(k_perm))) return PBS_ERR_INVALID_ARG;
+    if (kbar_sum && !aligned16(kbar_sum)) return PBS_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws)) return PBS_ERR_INVALID_ARG;
+    if (ws_bytes < select_ws_bytes(dm, kbar_sum == nullptr)) return PBS_ERR_WORKSPACE;
+  }
+  int *err = error_word();
+  cudaStream_t cs = (cudaStream_t)st;
+  double *qsum = (double *)ws;
+  const double *ksum = kbar_sum;
+  if (scored) {
+    cudaError_t e = launch_blocksum(dm, dm.b * dm.hq, q_or_qperm, qsum, cs);
+    if (e != cudaSuccess) return PBS_ERR_CUDA;
+    if (!kbar_sum) {
+      double *kbuf = qsum + (size_t)dm.b * dm.hq * dm.nb * dm.d;
+      e = launch_blocksum(dm, dm.b * dm.hkv, k_perm, kbuf, cs);
+      if (e != cudaSuccess) return PBS_ERR_CUDA;
+      ksum = kbuf;
+    }
+  }
+  return cuda_status(launch_select(dm, qsum, ksum, mode, param, resolve_sigma(scale, dm.d),
+                                   blk_idx, blk_cnt, blk_mask, err, cs));
+}
+
+pbs_status pbs_attn_fwd(const void *q_or_qperm, const void *k_perm, const void *v_perm,
+                        const int32_t *kpos, const int32_t *qpos, const int32_t *blk_idx,
+                        const int32_t *blk_cnt, void *out, float *lse, pbs_shape s, float scale,
+                        pbs_stream_t st) {
+  Dims dm;
+  pbs_status r = check_shape(s, &dm);
+  if (r != PBS_OK) return r;
+  if (empty(dm)) return PBS_OK;
+  if (!q_or_qperm || !k_perm || !v_perm || !blk_idx || !blk_cnt || !out)
+    return PBS_ERR_INVALID_ARG;
+  if (!aligned16(q_or_qperm) || !aligned16(k_perm) || !aligned16(v_perm) || !aligned16(out) ||
+      (kpos && !aligned16(kpos)) || (qpos && ((uintptr_t)qpos & 3u)) ||
+      ((uintptr_t)blk_idx & 3u) || ((uintptr_t)blk_cnt & 3u) || (lse && ((uintptr_t)lse & 3u)))
+    return PBS_ERR_INVALID_ARG;
+  int *err = error_word();
+  const float sigma = (float)resolve_sigma(scale, dm.d);
+  return cuda_status(launch_attn(dm, q_or_qperm, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt,
+                                 out, lse, sigma, err, (cudaStream_t)st));
+}
+
+pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out, pbs_shape s,
+                         pbs_stream_t st) {
+  Dims dm;
+  pbs_status r = check_shape(s, &dm);
+  if (r != PBS_OK) return r;
+  if (empty(dm)) return PBS_OK;
+  if (!out_perm || !out || !aligned16(out_perm) || !aligned16(out) ||
+      (qpos && ((uintptr_t)qpos & 3u)))
+    return PBS_ERR_INVALID_ARG;
+  cudaStream_t cs = (cudaStream_t)st;
+  if (!qpos) {
+    if (out == out_perm) return PBS_OK;
+    const size_t bytes = (size_t)dm.b * dm.hq * dm.n * dm.d * 2;
+    return cuda_status(cudaMemcpyAsync(out, out_perm, bytes, cudaMemcpyDeviceToDevice, cs));
+  }
+  if (out == out_perm) return PBS_ERR_INVALID_ARG;
+  return cuda_status(launch_unpermute(dm, out_perm, qpos, out, error_word(), cs));
+}
+
+pbs_status pbs_get_device_status(pbs_stream_t st, int *code) {
+  if (!code) return PBS_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)st) != cudaSuccess) return PBS_ERR_CUDA;
+  int *err = error_word();
+  if (!err) return PBS_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PBS_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return PBS_ERR_CUDA;
+  *code = v;
+  return PBS_OK;
+}
+
+const char *pbs_status_string(int status) {
+  switch (status) {
+    case PBS_OK: return "PBS_OK";
+    case PBS_ERR_INVALID_ARG: return "PBS_ERR_INVALID_ARG";
+    case PBS_ERR_UNSUPPORTED: return "PBS_ERR_UNSUPPORTED";
+    case PBS_ERR_CUDA: return "PBS_ERR_CUDA";
+    case PBS_ERR_TIMEOUT: return "PBS_ERR_TIMEOUT";
+    case PBS_ERR_DEVICE_ASSERT: return "PBS_ERR_DEVICE_ASSERT";
+    case PBS_ERR_WORKSPACE: return "PBS_ERR_WORKSPACE";
+    default: return "PBS_ERR_UNKNOWN";
+  }
+}
+
+const char *pbs_version(void) { return "pbs-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

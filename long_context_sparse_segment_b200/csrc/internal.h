@@ -1,0 +1,57 @@
+// Internal launcher interface of libpbs (not part of the public ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pbs {
+
+struct Dims {
+  int b, hq, hkv, n, d, B, S;
+  int G;    // hq / hkv
+  int nb;   // n / B
+  int spb;  // S / B
+  int nseg; // ceil(n / S)
+};
+
+// pass-1/2 importance scoring
+size_t score_ws_bytes(const Dims &dm);
+bool score_supported(const Dims &dm);
+cudaError_t launch_score(const Dims &dm, const void *q, const void *k, float *imp,
+                         float sigma, void *ws, int *err, cudaStream_t st);
+
+// segment sort (imp -> kpos) and the gather of K, V (and Q) by kpos
+cudaError_t launch_segsort(const Dims &dm, const float *imp, int32_t *kpos, int *err,
+                           cudaStream_t st);
+cudaError_t launch_gather(const Dims &dm, const int32_t *kpos, const void *k, const void *v,
+                          const void *q, void *kp, void *vp, void *qp, double *kbar, int *err,
+                          cudaStream_t st);
+
+// fp64 sums of every run of B rows: x [heads, n, d] bf16 -> out [heads, nb, d]
+cudaError_t launch_blocksum(const Dims &dm, int heads, const void *x, double *out,
+                            cudaStream_t st);
+
+// block lists from pooled sums
+size_t select_ws_bytes(const Dims &dm, bool need_kbar);
+cudaError_t launch_select(const Dims &dm, const double *qsum, const double *ksum, int mode,
+                          float param, double sigma, int32_t *idx, int32_t *cnt,
+                          uint8_t *mask, int *err, cudaStream_t st);
+
+// block-sparse forward
+cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const void *vp,
+                        const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
+                        const int32_t *cnt, void *out, float *lse, float sigma, int *err,
+                        cudaStream_t st);
+
+// the same forward on the legacy warp-MMA path
+cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const void *vp,
+                            const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
+                            const int32_t *cnt, void *out, float *lse, float sigma, int *err,
+                            cudaStream_t st);
+
+// out[qpos[p]] = out_perm[p]
+cudaError_t launch_unpermute(const Dims &dm, const void *op, const int32_t *qpos, void *out,
+                             int *err, cudaStream_t st);
+
+}  // namespace pbs

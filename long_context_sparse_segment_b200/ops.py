@@ -1,0 +1,172 @@
+"""PyTorch-facing calls of libpbs: argument marshalling only.
+
+Every step runs in the library's CUDA kernels; these functions only check
+tensor dtypes and devices, allocate outputs with torch, and pass raw device
+pointers plus the current CUDA stream through the C ABI (include/pbs.h).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import Shape, check, lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, name, dtype, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def shape_of(q, k, block, segment) -> Shape:
+    b, hq, n, d = q.shape
+    return Shape(b, hq, k.shape[1], n, d, block, segment)
+
+
+def workspace_bytes(shape: Shape, op: int) -> int:
+    return int(lib().pbs_workspace_bytes(shape, op))
+
+
+def _workspace(shape, op, device, ws=None):
+    need = workspace_bytes(shape, op)
+    if ws is not None and ws.numel() * ws.element_size() >= need:
+        return ws, need
+    return torch.empty(max(need, 16), dtype=torch.uint8, device=device), need
+
+
+def score(q, k, block, segment=None, scale=0.0, ws=None, out=None):
+    """Key importance imp [b, hkv, n] fp32 from the last query block."""
+    _need(q, "q", torch.bfloat16)
+    _need(k, "k", torch.bfloat16, q.device)
+    shp = shape_of(q, k, block, segment or block)
+    b, hkv, n, _ = k.shape
+    imp = out if out is not None else torch.empty(b, hkv, n, dtype=torch.float32, device=q.device)
+    ws, need = _workspace(shp, _lib.OP_SCORE, q.device, ws)
+    check(lib().pbs_score(_ptr(q), _ptr(k), _ptr(imp), shp, scale, _ptr(ws), need,
+                          _stream(q.device)), "pbs_score")
+    return imp
+
+
+def permute(imp, k, v, block, segment, q=None, kbar=True, hq=None):
+    """Segment-local order and gathers. Returns dict(kpos, k_perm, v_perm,
+    kbar_sum[, q_perm])."""
+    _need(imp, "imp", torch.float32)
+    _need(k, "k", torch.bfloat16, imp.device)
+    _need(v, "v", torch.bfloat16, imp.device)
+    b, hkv, n, d = k.shape
+    if q is not None:
+        _need(q, "q", torch.bfloat16, imp.device)
+        hq = q.shape[1]
+    shp = Shape(b, hq or hkv, hkv, n, d, block, segment)
+    out = {
+        "kpos": torch.empty(b, hkv, n, dtype=torch.int32, device=k.device),
+        "k_perm": torch.empty_like(k),
+        "v_perm": torch.empty_like(v),
+        "kbar_sum": (torch.empty(b, hkv, n // block, d, dtype=torch.float64, device=k.device)
+                     if kbar else None),
+        "q_perm": torch.empty_like(q) if q is not None else None,
+    }
+    check(lib().pbs_permute(_ptr(imp), _ptr(k), _ptr(v), _ptr(q), _ptr(out["k_perm"]),
+                            _ptr(out["v_perm"]), _ptr(out["q_perm"]), _ptr(out["kpos"]),
+                            _ptr(out["kbar_sum"]), shp, _stream(k.device)), "pbs_permute")
+    return out
+
+
+def select_blocks(q, k_perm, kbar_sum, block, segment, mode, param=0.0, scale=0.0, mask=False,
+                  ws=None, idx=None, cnt=None):
+    """Kept block lists: (blk_idx [b,hq,nb,nb] int32, blk_cnt [b,hq,nb] int32,
+    blk_mask [b,hq,nb,nb] uint8 or None)."""
+    _need(q, "q", torch.bfloat16)
+    if kbar_sum is not None:
+        _need(kbar_sum, "kbar_sum", torch.float64, q.device)
+    if k_perm is not None:
+        _need(k_perm, "k_perm", torch.bfloat16, q.device)
+    hkv = (k_perm if k_perm is not None else kbar_sum).shape[1]
+    b, hq, n, d = q.shape
+    shp = Shape(b, hq, hkv, n, d, block, segment)
+    nb = n // block
+    mode_id = _lib.SEL[mode] if isinstance(mode, str) else int(mode)
+    idx = idx if idx is not None else torch.empty(b, hq, nb, nb, dtype=torch.int32, device=q.device)
+    cnt = cnt if cnt is not None else torch.empty(b, hq, nb, dtype=torch.int32, device=q.device)
+    msk = torch.empty(b, hq, nb, nb, dtype=torch.uint8, device=q.device) if mask else None
+    ws, need = _workspace(shp, _lib.OP_SELECT, q.device, ws)
+    check(lib().pbs_select_blocks(_ptr(q), _ptr(k_perm), _ptr(kbar_sum), shp, mode_id, param,
+                                  scale, _ptr(idx), _ptr(cnt), _ptr(msk), _ptr(ws), need,
+                                  _stream(q.device)), "pbs_select_blocks")
+    return idx, cnt, msk
+
+
+def attn_fwd(q, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt, block, segment, scale=0.0,
+             lse=False, out=None):
+    """Block-sparse causal attention over the permuted keys: o [b,hq,n,d] bf16
+    (and lse [b,hq,n] fp32 when asked)."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_perm, "k_perm", torch.bfloat16, q.device)
+    _need(v_perm, "v_perm", torch.bfloat16, q.device)
+    for t, nm in ((kpos, "kpos"), (qpos, "qpos")):
+        if t is not None:
+            _need(t, nm, torch.int32, q.device)
+    _need(blk_idx, "blk_idx", torch.int32, q.device)
+    _need(blk_cnt, "blk_cnt", torch.int32, q.device)
+    shp = shape_of(q, k_perm, block, segment)
+    o = out if out is not None else torch.empty_like(q)
+    l = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if lse else None
+    check(lib().pbs_attn_fwd(_ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(kpos), _ptr(qpos),
+                             _ptr(blk_idx), _ptr(blk_cnt), _ptr(o), _ptr(l), shp, scale,
+                             _stream(q.device)), "pbs_attn_fwd")
+    return (o, l) if lse else o
+
+
+def unpermute(o_perm, qpos, hkv, block, segment, out=None):
+    """o[b, g, qpos[b, g/G, p]] = o_perm[b, g, p]."""
+    _need(o_perm, "o_perm", torch.bfloat16)
+    if qpos is not None:
+        _need(qpos, "qpos", torch.int32, o_perm.device)
+    b, hq, n, d = o_perm.shape
+    shp = Shape(b, hq, hkv, n, d, block, segment)
+    o = out if out is not None else torch.empty_like(o_perm)
+    check(lib().pbs_unpermute(_ptr(o_perm), _ptr(qpos), _ptr(o), shp, _stream(o_perm.device)),
+          "pbs_unpermute")
+    return o
+
+
+def device_status(device=None) -> int:
+    code = ctypes.c_int(0)
+    check(lib().pbs_get_device_status(_stream(device), ctypes.byref(code)), "pbs_get_device_status")
+    return code.value
+
+
+def pbs_attention(q, k, v, block, segment, mode="threshold", param=0.9, scale=0.0,
+                  permute_q=False, keep=False):
+    """The whole prefill path: score -> permute -> select -> attend ->
+    unpermute. Returns o [b, hq, n, d] bf16 in the natural query order, or a
+    dict with every intermediate when ``keep`` is true."""
+    imp = score(q, k, block, segment, scale)
+    perm = permute(imp, k, v, block, segment, q=q if permute_q else None, hq=q.shape[1])
+    q_used = perm["q_perm"] if permute_q else q
+    qpos = perm["kpos"] if permute_q else None
+    idx, cnt, _ = select_blocks(q_used, perm["k_perm"], perm["kbar_sum"], block, segment, mode,
+                                param, scale)
+    o_perm = attn_fwd(q_used, perm["k_perm"], perm["v_perm"], perm["kpos"], qpos, idx, cnt,
+                      block, segment, scale)
+    o = unpermute(o_perm, qpos, k.shape[1], block, segment) if permute_q else o_perm
+    if keep:
+        return dict(perm, imp=imp, idx=idx, cnt=cnt, o_perm=o_perm, o=o, qpos=qpos)
+    return o

@@ -224,6 +224,21 @@ def select_blocks(q_pooled, k_pooled, spb, mode, param, scale, group):
 # Step 4: block-sparse causal attention on the permuted sequence
 # (sciencestack.ai Figure 1 caption; gist.science "Methodik" 2 and 4)
 # --------------------------------------------------------------------------
+def attend_blocks(q, k_perm, v_perm, kpos, qpos, idx, cnt, block, blocks, scale=None):
+    """``attend`` for whole query blocks only: blocks is an iterable of
+    (batch, head, query block); returns [len(blocks), block, d]."""
+    hkv = k_perm.shape[1]
+    g_sz = q.shape[1] // hkv
+    sigma = resolve_scale(scale, q.shape[3])
+    blocks = list(blocks)
+    out = np.zeros((len(blocks), block, q.shape[3]))
+    for t, (bi, g, blk) in enumerate(blocks):
+        r = np.arange(blk * block, (blk + 1) * block)
+        out[t] = _attend_rows(q, k_perm, v_perm, kpos, qpos, idx, cnt, block, sigma, bi, g,
+                              g // g_sz, blk, r)
+    return out
+
+
 def attend(q, k_perm, v_perm, kpos, qpos, idx, cnt, block, scale=None, rows=None):
     """Output rows of the permuted block-sparse attention.
 

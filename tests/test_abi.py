@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry
+point of include/pbs.h, and rejects bad arguments before launching anything
+(none of these calls reaches a kernel, so no GPU is needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import long_context_sparse_segment_b200 as pbs
+from long_context_sparse_segment_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from long_context_sparse_segment_b200 import build
+        build.build()
+    return pbs.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "pbs.h")).read()
+    return set(re.findall(r"^\S[^;(]*?\b(pbs_\w+)\s*\(", text, flags=re.M))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = header_functions()
+    assert declared == set(_lib.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (pbs_\w+)", out))
+    assert declared <= exported
+
+
+def test_version_and_status_strings(lib):
+    assert b"sm_100a" in lib.pbs_version()
+    assert pbs.status_string(0) == "PBS_OK"
+    assert pbs.status_string(4) == "PBS_ERR_TIMEOUT"
+    assert pbs.status_string(99) == "PBS_ERR_UNKNOWN"
+
+
+GOOD = dict(batch=1, hq=8, hkv=2, n=1024, d=128, block=128, segment=256)
+
+
+def shape(**kw):
+    f = dict(GOOD, **kw)
+    return pbs.Shape(*(f[k] for k in ("batch", "hq", "hkv", "n", "d", "block", "segment")))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(hq=6, hkv=4), _lib.ERR_INVALID_ARG),         # hq not a multiple of hkv
+    (dict(d=96), _lib.ERR_UNSUPPORTED),
+    (dict(block=32), _lib.ERR_UNSUPPORTED),
+    (dict(segment=200), _lib.ERR_INVALID_ARG),         # S not a multiple of B
+    (dict(n=1000), _lib.ERR_INVALID_ARG),              # N not a multiple of B
+    (dict(n=-128), _lib.ERR_INVALID_ARG),
+    (dict(segment=16384), _lib.ERR_UNSUPPORTED),
+])
+def test_bad_shapes_are_rejected(lib, kw, code):
+    fake = ctypes.c_void_p(1 << 20)
+    s = shape(**kw)
+    assert lib.pbs_score(fake, fake, fake, s, 0.0, fake, 1 << 30, None) == code
+    assert lib.pbs_attn_fwd(fake, fake, fake, None, None, fake, fake, fake, None, s, 0.0,
+                            None) == code
+    assert lib.pbs_workspace_bytes(s, 0) == 0
+
+
+def test_null_and_misaligned_pointers(lib):
+    s = shape()
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    ws = pbs.workspace_bytes(s, _lib.OP_SCORE)
+    assert lib.pbs_score(None, fake, fake, s, 0.0, fake, ws, None) == _lib.ERR_INVALID_ARG
+    assert lib.pbs_score(odd, fake, fake, s, 0.0, fake, ws, None) == _lib.ERR_INVALID_ARG
+    assert lib.pbs_score(fake, fake, fake, s, 0.0, fake, ws - 1, None) == _lib.ERR_WORKSPACE
+    # q without q_perm, and in-place gathers
+    assert lib.pbs_permute(fake, fake, fake, fake, odd, odd, None, fake, None, s,
+                           None) == _lib.ERR_INVALID_ARG
+    assert lib.pbs_permute(fake, fake, fake, None, fake, fake, None, fake, None, s,
+                           None) == _lib.ERR_INVALID_ARG
+    assert lib.pbs_unpermute(fake, fake, fake, s, None) == _lib.ERR_INVALID_ARG
+
+
+def test_selection_arguments(lib):
+    s = shape()
+    fake = ctypes.c_void_p(1 << 20)
+    ws = pbs.workspace_bytes(s, _lib.OP_SELECT)
+    for mode, param in ((0, 0.0), (0, 1.5), (1, -0.1), (7, 0.5)):
+        assert lib.pbs_select_blocks(fake, fake, fake, s, mode, param, 0.0, fake, fake, None,
+                                     fake, ws, None) == _lib.ERR_INVALID_ARG
+    assert lib.pbs_select_blocks(fake, fake, None, s, 0, 0.9, 0.0, fake, fake, None, fake,
+                                 ws // 2, None) == _lib.ERR_WORKSPACE
+
+
+def test_empty_calls_launch_nothing(lib):
+    s = shape(n=0)
+    assert lib.pbs_score(None, None, None, s, 0.0, None, 0, None) == 0
+    assert lib.pbs_attn_fwd(None, None, None, None, None, None, None, None, None, s, 0.0,
+                            None) == 0
+    s = shape(batch=0)
+    assert lib.pbs_permute(None, None, None, None, None, None, None, None, None, s, None) == 0
+
+
+def test_workspace_sizes_grow_with_the_problem(lib):
+    a = pbs.workspace_bytes(shape(), _lib.OP_SELECT)
+    b = pbs.workspace_bytes(shape(n=2048), _lib.OP_SELECT)
+    assert b == 2 * a > 0
+    assert pbs.workspace_bytes(shape(), _lib.OP_ATTN) == 0

@@ -1,0 +1,197 @@
+"""GPU parity of every step of the path against the CPU oracle, through the
+C ABI, on seeded synthetic inputs (sizes the oracle finishes in seconds,
+spanning several tiles, with ragged segments and the degenerate cases).
+
+Split of the parity bar:
+  * score: fp32 importance within 1e-4 relative of the fp64 oracle;
+  * permute: the oracle's segment order applied to the GPU's own importance
+    equals the GPU kpos bit for bit; K', V' are exact gathers; the fp64 block
+    sums are exact;
+  * select: the oracle fed the GPU's permuted keys gives bit-identical lists
+    (decisions with a margin below 1e-12 are reported, not compared);
+  * forward: the oracle fed the GPU's kpos and lists is within max-abs 2e-2
+    and mean-abs 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import long_context_sparse_segment_b200 as pbs
+from long_context_sparse_segment_b200.workloads import WORKLOADS, Workload, make_inputs
+from oracle import pbs_oracle as orc
+from pbs_testutil import (assert_importance_close, assert_outputs_close, compare_lists, f64,
+                          i64)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny": WORKLOADS["tiny"],
+    # Llama-shaped GQA, reduced length
+    "gqa2k": Workload("gqa2k", 1, 8, 2, 2048, 128, 128, 512, "threshold", 0.9,
+                      "per_segment", 0.02),
+    # two batches, last segment shorter than S, top-k selection
+    "ragged": Workload("ragged", 2, 4, 2, 1280, 128, 128, 512, "topk_frac", 0.3,
+                       "per_segment", 0.02),
+    "d64_b128": Workload("d64_b128", 1, 4, 1, 1024, 64, 128, 256, "threshold", 0.7,
+                         "uniform", 0.05),
+    "d128_b64": Workload("d128_b64", 1, 4, 4, 1024, 128, 64, 256, "topk_frac", 0.25,
+                         "uniform", 0.05),
+    # S = B: one block per segment
+    "s_eq_b": Workload("s_eq_b", 1, 4, 2, 1024, 128, 128, 128, "threshold", 0.9,
+                       "uniform", 0.05),
+    # S = N: one segment, every block forced
+    "s_eq_n": Workload("s_eq_n", 1, 2, 1, 1024, 64, 64, 1024, "threshold", 0.5,
+                       "uniform", 0.05),
+}
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    return torch.device("cuda", 0)
+
+
+def inputs(w, dev):
+    q, k, v, _ = make_inputs(w)
+    return (q, k, v), (q.to(dev), k.to(dev), v.to(dev))
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_steps_against_oracle(name, dev):
+    w = CASES[name]
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    q64, k64, v64 = f64(q), f64(k), f64(v)
+
+    imp = pbs.score(qd, kd, B)
+    assert_importance_close(f64(imp), orc.score(q64, k64, B))
+
+    perm = pbs.permute(imp, kd, vd, B, S, hq=w.hq)
+    kpos = i64(perm["kpos"])
+    np.testing.assert_array_equal(kpos, orc.segment_order(f64(imp), S))
+    kp = perm["k_perm"]
+    assert torch.equal(kp.cpu(), torch.from_numpy(np.take_along_axis(
+        k.float().numpy(), kpos[..., None], axis=2)).to(torch.bfloat16))
+    assert torch.equal(perm["v_perm"].cpu(), torch.from_numpy(np.take_along_axis(
+        v.float().numpy(), kpos[..., None], axis=2)).to(torch.bfloat16))
+    np.testing.assert_array_equal(f64(perm["kbar_sum"]), orc.block_means(f64(kp), B) * B)
+
+    idx, cnt, mask = pbs.select_blocks(qd, kp, perm["kbar_sum"], B, S, w.mode, w.param,
+                                       mask=True)
+    ref_idx, ref_cnt, margin = orc.select_blocks(orc.block_means(q64, B),
+                                                 orc.block_means(f64(kp), B), S // B, w.mode,
+                                                 w.param, None, w.group)
+    assert compare_lists(idx, cnt, ref_idx, ref_cnt, margin) == 0
+    m = i64(mask)
+    for r in np.ndindex(*ref_cnt.shape):
+        assert m[r].sum() == ref_cnt[r]
+        assert np.all(m[r][ref_idx[r][:ref_cnt[r]]] == 1)
+
+    o = pbs.attn_fwd(qd, kp, perm["v_perm"], perm["kpos"], None, idx, cnt, B, S)
+    ref_o = orc.attend(q64, f64(kp), f64(perm["v_perm"]), kpos, None, i64(idx), i64(cnt), B)
+    assert_outputs_close(f64(o), ref_o, name)
+
+
+@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d128_b64"])
+@pytest.mark.parametrize("permute_q", [False, True])
+def test_end_to_end_against_oracle(name, permute_q, dev):
+    """The whole path against the oracle's own pipeline. The permutations may
+    differ only inside runs of near-equal importance; outputs must agree."""
+    w = CASES[name]
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    res = pbs.pbs_attention(qd, kd, vd, w.block, w.segment, w.mode, w.param,
+                            permute_q=permute_q, keep=True)
+    ref = orc.pbs_attention(f64(q), f64(k), f64(v), w.block, w.segment, w.mode, w.param,
+                            permute_q=permute_q)
+    diff = (i64(res["kpos"]) != ref["kpos"]).mean()
+    assert diff < 0.05, f"{diff:.3%} of key slots differ"
+    assert_outputs_close(f64(res["o"]), ref["o"], name)
+
+
+def test_permuted_query_mode_steps(dev):
+    w = CASES["gqa2k"]
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    imp = pbs.score(qd, kd, B)
+    perm = pbs.permute(imp, kd, vd, B, S, q=qd)
+    kpos = i64(perm["kpos"])
+    qpos = np.repeat(kpos, w.group, axis=1)
+    assert torch.equal(perm["q_perm"].cpu(), torch.from_numpy(np.take_along_axis(
+        q.float().numpy(), qpos[..., None], axis=2)).to(torch.bfloat16))
+    idx, cnt, _ = pbs.select_blocks(perm["q_perm"], perm["k_perm"], perm["kbar_sum"], B, S,
+                                    w.mode, w.param)
+    o_perm = pbs.attn_fwd(perm["q_perm"], perm["k_perm"], perm["v_perm"], perm["kpos"],
+                          perm["kpos"], idx, cnt, B, S)
+    ref = orc.attend(f64(perm["q_perm"]), f64(perm["k_perm"]), f64(perm["v_perm"]), kpos, qpos,
+                     i64(idx), i64(cnt), B)
+    assert_outputs_close(f64(o_perm), ref, "q-permuted forward")
+    o = pbs.unpermute(o_perm, perm["kpos"], w.hkv, B, S)
+    assert torch.equal(o.cpu(), torch.from_numpy(np.ascontiguousarray(
+        orc.unpermute(f64(o_perm), qpos))).to(torch.bfloat16))
+
+
+def test_all_blocks_equals_dense_causal(dev):
+    """Theorem 3.3 on the GPU path: with every admissible block kept, the
+    permuted forward equals plain causal attention (identity order, blocks
+    J <= I) on the same kernel."""
+    w = CASES["gqa2k"]
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    imp = pbs.score(qd, kd, B)
+    perm = pbs.permute(imp, kd, vd, B, S, hq=w.hq)
+    idx, cnt, _ = pbs.select_blocks(qd, perm["k_perm"], perm["kbar_sum"], B, S, "all")
+    o_all = pbs.attn_fwd(qd, perm["k_perm"], perm["v_perm"], perm["kpos"], None, idx, cnt, B, S)
+    didx, dcnt, _ = pbs.select_blocks(qd, kd, None, B, S, "dense_causal")
+    o_dense = pbs.attn_fwd(qd, kd, vd, None, None, didx, dcnt, B, S)
+    ref = orc.dense_causal(f64(q), f64(k), f64(v))
+    assert_outputs_close(f64(o_all), ref, "all blocks")
+    assert_outputs_close(f64(o_dense), ref, "dense causal")
+    assert_outputs_close(f64(o_all), f64(o_dense), "all vs dense")
+
+
+def test_exact_importance_ties_keep_lower_index(dev):
+    w = CASES["gqa2k"]
+    (_, k, v), (_, kd, vd) = inputs(w, dev)
+    g = torch.Generator().manual_seed(5)
+    imp = torch.randint(0, 4, (1, 2, 2048), generator=g).float() / 8   # heavy ties
+    perm = pbs.permute(imp.to(dev), kd, vd, 128, 512, hq=8)
+    np.testing.assert_array_equal(i64(perm["kpos"]), orc.segment_order(imp.double().numpy(), 512))
+
+
+def test_lse_output(dev):
+    w = CASES["d128_b64"]
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    idx, cnt, _ = pbs.select_blocks(qd, kd, None, w.block, w.segment, "dense_causal")
+    o, lse = pbs.attn_fwd(qd, kd, vd, None, None, idx, cnt, w.block, w.segment, lse=True)
+    q64, k64 = f64(q), f64(k)
+    sigma = 1.0 / np.sqrt(w.d)
+    for g in range(w.hq):
+        logits = sigma * q64[0, g] @ k64[0, g].T
+        logits = np.where(np.tril(np.ones((w.n, w.n), bool)), logits, -np.inf)
+        mx = logits.max(1)
+        want = mx + np.log(np.exp(logits - mx[:, None]).sum(1))
+        np.testing.assert_allclose(f64(lse)[0, g], want, atol=2e-3)
+
+
+def test_deterministic(dev):
+    w = CASES["ragged"]
+    _, (qd, kd, vd) = inputs(w, dev)
+    a = pbs.pbs_attention(qd, kd, vd, w.block, w.segment, w.mode, w.param, keep=True)
+    b = pbs.pbs_attention(qd, kd, vd, w.block, w.segment, w.mode, w.param, keep=True)
+    for key in ("imp", "kpos", "k_perm", "kbar_sum", "cnt", "o"):
+        assert torch.equal(a[key], b[key]), key
+
+
+def test_empty_sequence(dev):
+    q = torch.empty(1, 4, 0, 128, dtype=torch.bfloat16, device=dev)
+    k = torch.empty(1, 2, 0, 128, dtype=torch.bfloat16, device=dev)
+    o = pbs.pbs_attention(q, k, k, 128, 512)
+    assert o.shape == q.shape
+
+
+def test_device_status_is_clean(dev):
+    w = CASES["tiny"]
+    _, (qd, kd, vd) = inputs(w, dev)
+    pbs.pbs_attention(qd, kd, vd, w.block, w.segment)
+    assert pbs.device_status() == 0
