@@ -102,6 +102,31 @@ pbs_status pbs_score(const void *q, const void *k, float *imp, pbs_shape s,
                      float scale, void *ws, size_t ws_bytes, pbs_stream_t st);
 
 /*
+ * pbs_score_static - pbs_score for callers that cannot allocate device memory.
+ * The paper has no counterpart: this is a deployment variant of pbs_score.
+ *
+ * Callers such as a plugin inside an inference engine that owns every
+ * device allocation (and forbids cudaMalloc), or a latency-critical loop
+ * that cannot take cudaMalloc's implicit synchronisation, cannot provide
+ * pbs_score's workspace. This call computes the same importance with its
+ * scratch in a fixed array of PBS_SCORE_STATIC_SCRATCH_BYTES inside the
+ * library, held on every GPU that loads the library until the process
+ * exits. It allocates nothing; the caller still passes q, k and imp.
+ *
+ * - Shapes whose scoring scratch (pbs_workspace_bytes(s, PBS_OP_SCORE))
+ *   exceeds the array return PBS_ERR_WORKSPACE and launch nothing.
+ * - The first call on a device (with that device current) looks up the
+ *   array's device address; make it before any stream capture.
+ * - All calls share the array and it keeps the previous call's contents
+ *   (nothing in it needs to start at zero). Calls that overlap on the GPU,
+ *   from several streams or threads, race on it: serialise them.
+ * Other arguments, errors and results: as pbs_score.
+ */
+#define PBS_SCORE_STATIC_SCRATCH_BYTES (4u << 20)
+pbs_status pbs_score_static(const void *q, const void *k, float *imp, pbs_shape s,
+                            float scale, pbs_stream_t st);
+
+/*
  * pbs_permute - segment-local key permutation and gather.
  * Source: gist.science summary, "Methodik" 2 (segmented permutation: only
  * inside contiguous segments of S tokens, segment order kept) and 3

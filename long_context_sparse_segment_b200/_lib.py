@@ -16,7 +16,7 @@ SEL = {"threshold": 0, "topk_frac": 1, "all": 2, "dense_causal": 3}
 OP_SCORE, OP_PERMUTE, OP_SELECT, OP_ATTN, OP_UNPERMUTE = range(5)
 
 # every entry point declared in include/pbs.h
-EXPORTS = ("pbs_workspace_bytes", "pbs_score", "pbs_permute", "pbs_select_blocks",
+EXPORTS = ("pbs_workspace_bytes", "pbs_score", "pbs_score_static", "pbs_permute", "pbs_select_blocks",
            "pbs_attn_fwd", "pbs_unpermute", "pbs_get_device_status", "pbs_status_string",
            "pbs_version")
 
@@ -37,6 +37,7 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 _SIGS = {
     "pbs_workspace_bytes": (_sz, [Shape, _i]),
     "pbs_score": (_i, [_vp, _vp, _vp, Shape, _f, _vp, _sz, _vp]),
+    "pbs_score_static": (_i, [_vp, _vp, _vp, Shape, _f, _vp]),
     "pbs_permute": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, Shape, _vp]),
     "pbs_select_blocks": (_i, [_vp, _vp, _vp, Shape, _i, _f, _f, _vp, _vp, _vp, _vp, _sz, _vp]),
     "pbs_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, Shape, _f, _vp]),
