@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--config", default="llama128k", choices=sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="time the steps only (no dense, end-to-end or CPU legs), for ncu")
     return ap.parse_args()
 
 
@@ -263,8 +265,11 @@ def gpu_arm(args):
     peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     attn_tflops = flops_per_step / len(layers) / (attn_launch_ms * 1e-3) / 1e12
 
-    dense_ms, dense_blocks = time_dense(layers[0])
-    e2e_ms, h2d, d2h = e2e_run(w, layers, max(1, args.e2e_steps))
+    if args.profile:
+        dense_ms, dense_blocks, e2e_ms, h2d, d2h = float("nan"), float("nan"), float("nan"), 0, 0
+    else:
+        dense_ms, dense_blocks = time_dense(layers[0])
+        e2e_ms, h2d, d2h = e2e_run(w, layers, max(1, args.e2e_steps))
     e2e_value = flops_per_step * world / (e2e_ms * 1e-3) / 1e12
     if dist:
         t = torch.tensor([e2e_ms], device=dev)
@@ -281,7 +286,7 @@ def gpu_arm(args):
                    "d": w.d, "block": w.block, "segment": w.segment, "layers": w.layers,
                    "selection": f"{w.mode} {w.param}", "l2": "inputs larger than L2",
                    "parallelism": f"replicas x{world}"},
-        "density": round(total_blocks / max(1.0, dense_blocks * len(layers)), 4),
+        "density": round(total_blocks / (len(layers) * w.batch * w.hq * w.nb * (w.nb + 1) / 2), 4),
         "breakdown_ms": {n: round(v, 4) for n, v in per.items()},
         "dense_attn_ms": round(dense_ms * len(layers), 4),
         "speedup_vs_dense": {"attn": round(dense_ms / attn_launch_ms, 3),
@@ -295,7 +300,7 @@ def gpu_arm(args):
                      "frac": round(attn_tflops / peak, 4), "peak_kind":
                      f"{pk_kind} bf16 dense, sustained", "traffic": traffic_for(w)},
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.profile):
         line["cpu_baseline"] = cpu_baseline(w, layers[0], total_blocks / len(layers))
     if rank == 0:
         print(json.dumps(line), flush=True)
