@@ -232,8 +232,11 @@ pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out,
 /*
  * Synchronises `st`, returns in *code the current device's error word
  * (a pbs_status; PBS_OK when no kernel reported a problem) and clears it.
+ * `detail` (nullable) receives a diagnostic: for PBS_ERR_TIMEOUT the place
+ * of the wait that ran out (tens digit: 1 K' loader, 2 V' loader, 3 MMA
+ * issuer, 4 softmax; units digit: which wait), else 0.
  */
-pbs_status pbs_get_device_status(pbs_stream_t st, int *code);
+pbs_status pbs_get_device_status(pbs_stream_t st, int *code, int *detail);
 
 /* Static, human-readable name of a status. */
 const char *pbs_status_string(int status);

@@ -42,7 +42,7 @@ _SIGS = {
     "pbs_select_blocks": (_i, [_vp, _vp, _vp, Shape, _i, _f, _f, _vp, _vp, _vp, _vp, _sz, _vp]),
     "pbs_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, Shape, _f, _vp]),
     "pbs_unpermute": (_i, [_vp, _vp, _vp, Shape, _vp]),
-    "pbs_get_device_status": (_i, [_vp, ctypes.POINTER(_i)]),
+    "pbs_get_device_status": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "pbs_status_string": (ctypes.c_char_p, [_i]),
     "pbs_version": (ctypes.c_char_p, []),
 }

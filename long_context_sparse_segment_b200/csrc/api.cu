@@ -12,8 +12,9 @@
 
 namespace pbs {
 
-// One error word per device: kernels record the first problem they meet.
-__device__ int g_error_word;
+// One error word per device: kernels record the first problem they meet in
+// [0] and, for a wait that ran out, the place of that wait in [1].
+__device__ int g_error_word[2];
 
 namespace {
 
@@ -199,17 +200,18 @@ pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out, p
   return cuda_status(launch_unpermute(dm, out_perm, qpos, out, error_word(), cs));
 }
 
-pbs_status pbs_get_device_status(pbs_stream_t st, int *code) {
+pbs_status pbs_get_device_status(pbs_stream_t st, int *code, int *detail) {
   if (!code) return PBS_ERR_INVALID_ARG;
   if (cudaStreamSynchronize((cudaStream_t)st) != cudaSuccess) return PBS_ERR_CUDA;
   int *err = error_word();
   if (!err) return PBS_ERR_CUDA;
-  int v = 0;
-  if (cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PBS_ERR_CUDA;
-  const int zero = 0;
-  if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+  int v[2] = {0, 0};
+  if (cudaMemcpy(v, err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return PBS_ERR_CUDA;
+  const int zero[2] = {0, 0};
+  if (cudaMemcpy(err, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
     return PBS_ERR_CUDA;
-  *code = v;
+  *code = v[0];
+  if (detail) *detail = v[1];
   return PBS_OK;
 }
 

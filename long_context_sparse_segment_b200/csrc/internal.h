@@ -44,6 +44,13 @@ cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const voi
                         const int32_t *cnt, void *out, float *lse, float sigma, int *err,
                         cudaStream_t st);
 
+// the forward on the tcgen05 tensor cores (B = 128, d in {64, 128})
+bool attn_tc_supported(const Dims &dm);
+cudaError_t launch_attn_tc(const Dims &dm, const void *q, const void *kp, const void *vp,
+                           const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
+                           const int32_t *cnt, void *out, float *lse, float sigma, int *err,
+                           int fault, cudaStream_t st);
+
 // the same forward on the legacy warp-MMA path
 cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,

@@ -147,10 +147,13 @@ def unpermute(o_perm, qpos, hkv, block, segment, out=None):
     return o
 
 
-def device_status(device=None) -> int:
-    code = ctypes.c_int(0)
-    check(lib().pbs_get_device_status(_stream(device), ctypes.byref(code)), "pbs_get_device_status")
-    return code.value
+def device_status(device=None, detail=False):
+    """Synchronise, read and clear the device error word: the pbs status code
+    (0 = no kernel reported a problem), plus the diagnostic detail if asked."""
+    code, where = ctypes.c_int(0), ctypes.c_int(0)
+    check(lib().pbs_get_device_status(_stream(device), ctypes.byref(code), ctypes.byref(where)),
+          "pbs_get_device_status")
+    return (code.value, where.value) if detail else code.value
 
 
 def pbs_attention(q, k, v, block, segment, mode="threshold", param=0.9, scale=0.0,

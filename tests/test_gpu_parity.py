@@ -195,3 +195,26 @@ def test_device_status_is_clean(dev):
     _, (qd, kd, vd) = inputs(w, dev)
     pbs.pbs_attention(qd, kd, vd, w.block, w.segment)
     assert pbs.device_status() == 0
+
+
+@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128"])
+def test_tensor_core_and_warp_mma_forwards_agree(name, dev, monkeypatch):
+    """The tcgen05 forward and the warp-MMA forward on the same lists, each
+    against the oracle."""
+    w = CASES[name]
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    imp = pbs.score(qd, kd, B)
+    perm = pbs.permute(imp, kd, vd, B, S, hq=w.hq)
+    idx, cnt, _ = pbs.select_blocks(qd, perm["k_perm"], perm["kbar_sum"], B, S, w.mode, w.param)
+    args = (qd, perm["k_perm"], perm["v_perm"], perm["kpos"], None, idx, cnt, B, S)
+    o_tc, lse_tc = pbs.attn_fwd(*args, lse=True)
+    monkeypatch.setenv("PBS_FORWARD", "mma")
+    o_mma, lse_mma = pbs.attn_fwd(*args, lse=True)
+    monkeypatch.delenv("PBS_FORWARD")
+    ref = orc.attend(f64(q), f64(perm["k_perm"]), f64(perm["v_perm"]), i64(perm["kpos"]), None,
+                     i64(idx), i64(cnt), B)
+    assert_outputs_close(f64(o_tc), ref, "tcgen05")
+    assert_outputs_close(f64(o_mma), ref, "warp mma")
+    np.testing.assert_allclose(f64(lse_tc), f64(lse_mma), atol=1e-3)
+    assert pbs.device_status() == 0
