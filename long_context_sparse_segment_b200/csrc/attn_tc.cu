@@ -233,13 +233,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float s[kBN];
       {
-        uint32_t r[32];
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(tS, r0);
+        tmem_ld32(tS + 32, r1);
+        tmem_ld32(tS + 64, r2);
+        tmem_ld32(tS + 96, r3);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-          tmem_ld32(tS + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) {
+          s[e] = __uint_as_float(r0[e]);
+          s[32 + e] = __uint_as_float(r1[e]);
+          s[64 + e] = __uint_as_float(r2[e]);
+          s[96 + e] = __uint_as_float(r3[e]);
         }
       }
       if (diag) {
@@ -262,9 +267,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (J * kBN + c > qp) s[c] = -INFINITY;
         }
       }
-      float mx = s[0];
+      // row max as 8 independent chains (one warp per scheduler: no other
+      // warp hides a 128-long dependent chain)
+      float m8[8];
 #pragma unroll
-      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+      for (int t = 0; t < 8; ++t) m8[t] = s[t];
+#pragma unroll
+      for (int c = 8; c < kBN; c += 8)
+#pragma unroll
+        for (int t = 0; t < 8; ++t) m8[t] = fmaxf(m8[t], s[c + t]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float mxs = mx * sl2;
       float alpha = 1.f;
       if (mxs > m_used + kRescaleLog2) {
@@ -273,21 +286,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float mu = m_used == -INFINITY ? 0.f : m_used;
       __syncwarp();  // reconverge after the per-row mask before the aligned stores
-      float sum = 0.f;
+      // p = 2^(s * sigma * log2(e) - m): packed fp32x2 FMA, the hardware
+      // exp2, four packed partial sums; P goes to TMEM as bf16 pairs over
+      // the first 64 columns of this S buffer.
+      const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-mu, -mu);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = exp2f(fmaf(s[c * 32 + 2 * e], sl2, -mu));
-          const float p1 = exp2f(fmaf(s[c * 32 + 2 * e + 1], sl2, -mu));
-          sum += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
+          const float2 x =
+              __ffma2_rn(make_float2(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]), scale2, neg_m2);
+          // 5 of every 16 pairs on the FMA pipe, the rest on MUFU
+          const float2 p = (e % 3 == 2) ? exp2_poly2(x)
+                                        : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          acc[e & 3] = __fadd2_rn(acc[e & 3], p);
+          pk[e] = pack_bf16(p.x, p.y);
         }
         tmem_st16(tS + c * 16, pk);
       }
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 a = __fadd2_rn(a01, a23);
       tmem_wait_st();
-      l = l * alpha + sum;
+      l = l * alpha + (a.x + a.y);
       if (j >= 1) {
         if (!mbar_wait_warp(&bar->o_ready, (j - 1) & 1, s_abort, err, 43)) {
           ok = false;

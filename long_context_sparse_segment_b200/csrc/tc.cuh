@@ -76,6 +76,40 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// The hardware base-2 exponential (MUFU), flushing subnormals: ex2(-inf) = 0.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x for a pair of floats on the FMA pipe, to take load off the MUFU unit.
+// Range reduction: adding 1.5 * 2^23 rounds x to the nearest integer n in the
+// low mantissa bits (round-to-nearest), so f = x - n lies in [-1/2, 1/2];
+// 2^f comes from a cubic fitted here by iteratively reweighted least squares
+// on the relative error (max relative error 7.5e-5 in fp32, far below the
+// bf16 rounding of P); 2^n is applied by adding n to the exponent field.
+// x is clamped to >= -125 so the result stays a normal float (masked
+// entries give ~2^-125 instead of 0, negligible against a row sum >= 1).
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.055171769112348557f;
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, magic);
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 p = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
+  p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
                                             int x, int y) {
