@@ -67,6 +67,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   }
 }
 
+// One arrival per warp on an mbarrier that counts warps: the warp's lanes
+// synchronise (ordering their earlier writes and fenced tcgen05 operations
+// before the arrival), then lane 0 arrives. 256 per-thread arrivals on one
+// barrier word would serialise in shared memory.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
 // The same wait taken by all 32 lanes of a warp: the result is made
 // uniform and the warp is reconverged, so that the .sync.aligned tcgen05
 // instructions that follow run on a converged warp.
@@ -192,6 +201,19 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// The same descriptor split in its two 32-bit words, for issue loops that
+// step through tiles with one add: lo = address >> 4 | (LBO >> 4) << 16,
+// hi = SBO >> 4 | version 1 << 14 | SWIZZLE_128B << 29.
+__device__ __forceinline__ uint32_t sw128_desc_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sw128_desc_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint64_t desc_words(uint32_t lo, uint32_t hi) {
+  return ((uint64_t)hi << 32) | lo;
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B.
