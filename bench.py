@@ -62,6 +62,28 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+RANK_SEED_STRIDE = 1000  # rank r draws its replica's inputs with seed + 1000 r
+
+
+def rank_seed_offset(rank):
+    return RANK_SEED_STRIDE * rank
+
+
+def job_throughput(flops_rank, ms_rank, dist=None, device="cpu"):
+    """Whole-job TFLOP/s: the flops of all ranks over the slowest rank's time.
+
+    Returns (TFLOP/s, slowest ms, total flops). Every rank must call it (it
+    holds two collectives when dist is given)."""
+    if dist is None:
+        return flops_rank / (ms_rank * 1e-3) / 1e12, ms_rank, flops_rank
+    t = torch.tensor([ms_rank], dtype=torch.float64, device=device)
+    f = torch.tensor([flops_rank], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(f, op=dist.ReduceOp.SUM)
+    ms, flops = float(t.item()), float(f.item())
+    return flops / (ms * 1e-3) / 1e12, ms, flops
+
+
 def block_flops(w, total_blocks):
     return 4.0 * w.block * w.block * w.d * total_blocks
 
@@ -222,7 +244,7 @@ def gpu_arm(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     w = WORKLOADS[args.config]
-    layers = [Layer(w, dev, l, seed_offset=1000 * rank) for l in range(w.layers)]
+    layers = [Layer(w, dev, l, seed_offset=rank_seed_offset(rank)) for l in range(w.layers)]
     torch.cuda.synchronize()
 
     # warm-up (also fixes the kept-block counts of this input)
@@ -255,12 +277,7 @@ def gpu_arm(args):
     ms = start.elapsed_time(stop) / args.steps
     per = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) / args.steps for n in names}
     attn_launch_ms = per["attn"] / len(layers)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-
-    value = flops_per_step * world / (ms * 1e-3) / 1e12
+    value, ms, _ = job_throughput(flops_per_step, ms, dist, dev)
     pk, pk_kind = peaks()
     peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     attn_tflops = flops_per_step / len(layers) / (attn_launch_ms * 1e-3) / 1e12
@@ -270,12 +287,7 @@ def gpu_arm(args):
     else:
         dense_ms, dense_blocks = time_dense(layers[0])
         e2e_ms, h2d, d2h = e2e_run(w, layers, max(1, args.e2e_steps))
-    e2e_value = flops_per_step * world / (e2e_ms * 1e-3) / 1e12
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-        e2e_value = flops_per_step * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value, e2e_ms, _ = job_throughput(flops_per_step, e2e_ms, dist, dev)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,

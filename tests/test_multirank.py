@@ -1,0 +1,70 @@
+"""Host-side logic of the N > 1 bench path, on two gloo ranks on the CPU.
+
+Under torchrun every rank runs its own replica of the workload (the path's
+units are independent, so no collective touches the data). What the ranks
+share is the reporting: the whole-job throughput is all ranks' work over the
+slowest rank's time, and every rank draws different inputs.
+"""
+import datetime
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    from long_context_sparse_segment_b200.workloads import WORKLOADS, make_inputs
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        flops = 1e12 * (rank + 1)
+        ms = 10.0 * (rank + 1)
+        value, ms_max, total = bench.job_throughput(flops, ms, dist, "cpu")
+        w = WORKLOADS["tiny"]
+        q, _, _, _ = make_inputs(w, seed=w.seed + bench.rank_seed_offset(rank))
+        digests = [None] * world
+        dist.all_gather_object(digests, float(q.float().sum()))
+        out.put((rank, value, ms_max, total, digests))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_report_whole_job_throughput_over_distinct_replicas():
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [out.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, value, ms_max, total, digests in results:
+        assert ms_max == 20.0                      # the slowest rank
+        assert total == 3e12                       # both ranks' work
+        assert value == pytest.approx(150.0)       # 3e12 flop / 20 ms
+        assert digests[0] != digests[1]            # replicas draw different inputs
+
+
+def test_single_process_throughput_needs_no_collective():
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    assert bench.job_throughput(2e12, 4.0) == (500.0, 4.0, 2e12)
+    assert bench.rank_seed_offset(0) == 0 and bench.rank_seed_offset(3) == 3000
