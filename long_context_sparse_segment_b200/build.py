@@ -17,7 +17,8 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpbs.so")
 
-SOURCES = ["api.cu", "score.cu", "score_static.cu", "permute.cu", "select.cu", "attn_mma.cu", "attn_tc.cu"]
+SOURCES = ["api.cu", "score.cu", "score_static.cu", "permute.cu", "select.cu", "attn_mma.cu", "attn_tc.cu",
+           "score_tc.cu", "tmap.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
          "--expt-relaxed-constexpr"]

@@ -28,7 +28,6 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -453,47 +452,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-  static EncodeTiled fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  });
-  return fn;
-}
-
-// [rows, d] bf16 rows, 128 x 64 boxes with the 128-byte swizzle.
-bool make_map(CUtensorMap *map, const void *ptr, uint64_t rows, int d) {
-  EncodeTiled enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t run(const Dims &dm, const void *q, const void *kp, const void *vp,
                 const int32_t *kpos, const int32_t *qpos, const int32_t *idx, const int32_t *cnt,
                 void *out, float *lse, float sigma, int *err, int fault, cudaStream_t st) {
   CUtensorMap mk, mv;
-  if (!make_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D) ||
-      !make_map(&mv, vp, (uint64_t)dm.b * dm.hkv * dm.n, D))
+  if (!make_tile_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D, 128) ||
+      !make_tile_map(&mv, vp, (uint64_t)dm.b * dm.hkv * dm.n, D, 128))
     return cudaErrorInvalidValue;
   const size_t smem = Cfg<D>::smem;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>,

@@ -21,6 +21,12 @@ bool score_supported(const Dims &dm);
 cudaError_t launch_score(const Dims &dm, const void *q, const void *k, float *imp,
                          float sigma, void *ws, int *err, cudaStream_t st);
 
+// the same two passes on the tcgen05 tensor cores (G*B a multiple of 128, <= 512)
+bool score_tc_supported(const Dims &dm);
+size_t score_tc_ws_bytes(const Dims &dm);
+cudaError_t launch_score_tc(const Dims &dm, const void *q, const void *k, float *imp,
+                            float sigma, void *ws, int *err, cudaStream_t st);
+
 // segment sort (imp -> kpos) and the gather of K, V (and Q) by kpos
 cudaError_t launch_segsort(const Dims &dm, const float *imp, int32_t *kpos, int *err,
                            cudaStream_t st);

@@ -15,6 +15,8 @@
 //           and the result is deterministic.
 // Logits are kept in the log2 domain: s = (q . k) * sigma * log2(e).
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -250,7 +252,9 @@ cudaError_t run(const Dims &dm, const void *q, const void *k, float *imp, float 
 size_t score_ws_bytes(const Dims &dm) {
   const size_t R = (size_t)dm.G * dm.B;
   const size_t bh = (size_t)dm.b * dm.hkv;
-  return (bh * score_splits(dm) * R + bh * R) * sizeof(float2);
+  const size_t mma = (bh * score_splits(dm) * R + bh * R) * sizeof(float2);
+  const size_t tc = score_tc_supported(dm) ? score_tc_ws_bytes(dm) : 0;
+  return mma > tc ? mma : tc;
 }
 
 bool score_supported(const Dims &dm) {
@@ -259,9 +263,14 @@ bool score_supported(const Dims &dm) {
          (dm.d == 64 ? score_smem<64>(R) : score_smem<128>(R)) <= 227 * 1024;
 }
 
+// The tcgen05 kernel serves G*B in {128, 256, 384, 512}; the warp-MMA
+// kernel every other supported shape. PBS_SCORE=mma selects the warp-MMA
+// kernel for every shape (a diagnostic switch for comparing the two).
 cudaError_t launch_score(const Dims &dm, const void *q, const void *k, float *imp, float sigma,
                          void *ws, int *err, cudaStream_t st) {
-  (void)err;
+  const char *sel = getenv("PBS_SCORE");
+  if (score_tc_supported(dm) && !(sel && strcmp(sel, "mma") == 0))
+    return launch_score_tc(dm, q, k, imp, sigma, ws, err, st);
   if (dm.d == 64) return run<64>(dm, q, k, imp, sigma, ws, st);
   return run<128>(dm, q, k, imp, sigma, ws, st);
 }

@@ -1,0 +1,410 @@
+// pbs_score on the sm_100a tensor cores (tcgen05 MMA, TMEM, TMA).
+//
+// "Sparser Block-Sparse Attention via Token Permutation", gist.science
+// summary, "Methodik" 3 ("Proxy-Bewertung"): the importance of a key is the
+// mean softmax probability the last query block gives it. For each (batch,
+// KV head) the R = G*B probe rows are the last B rows of the G query heads
+// that share the KV head; each row's softmax runs over all n keys (causal
+// inside the last block), so two passes over K are made. A CTA owns a
+// contiguous range of 128-key tiles of one (batch, KV head) and keeps the
+// probe rows Q_r (R x d) in shared memory.
+//
+// The two passes use opposite operand roles so that every reduction is
+// local to a thread, with no shuffles:
+//   pass 1: D = Q_w K_t^T, Q rows on the MMA's M side: the TMEM lane is a
+//           probe row, its columns are keys. Each thread keeps its row's
+//           running max and sum of exp2 -> partial (m, l) per (row, CTA).
+//   combine: per row, M = max m, L = sum l 2^(m - M); off = M + log2 L.
+//   pass 2: D = K_t Q_w^T, keys on the M side: the TMEM lane is a key, its
+//           columns are probe rows. p = 2^(s - off_r) summed over the
+//           thread's columns; the R/128 row groups' partial sums of a key
+//           are added in a fixed order -> imp = sum / R. Deterministic, no
+//           atomics.
+// Logits are in log2 units: s = (q . k) sigma log2(e).
+//
+// Roles (R/128 = W row groups; 128 W + 64 threads):
+//   warps 0 .. 4W-1   one warpgroup per 128-column TMEM slice w (probe rows
+//                     128w .. 128w+127); thread = TMEM lane;
+//   warp 4W, lane 0   TMA: the probe rows once, then K tiles into a ring;
+//   warp 4W+1, lane 0 tcgen05.mma issue: per K tile, one 128 x 128 x d
+//                     product per slice, each released as soon as its
+//                     warpgroup has read the slice into registers.
+// Every mbarrier wait is bounded (PBS_ERR_TIMEOUT, the CTA drains and exits).
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace pbs {
+namespace {
+
+using bf16 = __nv_bfloat16;
+using namespace tc;
+
+constexpr int kKT = 128;   // keys per tile
+constexpr int kMaxW = 4;   // R <= 512
+constexpr int kMaxKS = 4;  // K ring depth (upper bound)
+
+template <int D>
+struct SCfg {
+  static constexpr int H = D / 64;                         // 64-column boxes per row
+  static constexpr uint32_t TILE = 128u * D * 2;           // bytes of one 128-row tile
+  static constexpr uint32_t HALF = 128u * 128;             // bytes of one 64-column box
+  static constexpr int KS = D == 128 ? 2 : 4;              // K ring depth
+  static size_t smem(int R) {
+    return 1024 + (size_t)(R / 128) * TILE + (size_t)KS * TILE + sizeof(uint64_t) * 32 +
+           (size_t)R * 4 + 2 * kMaxW * 128 * 4 + 16;
+  }
+};
+
+struct SBars {
+  uint64_t q_full, k_full[kMaxKS], k_empty[kMaxKS], s_full[kMaxW], s_free[kMaxW], mma_done;
+};
+static_assert(sizeof(SBars) <= sizeof(uint64_t) * 32, "barrier block");
+
+__device__ __forceinline__ void softmax_bar(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+template <int D, int PASS>
+__global__ void __launch_bounds__(kMaxW * 128 + 64, 1)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmK, float *__restrict__ imp,
+                    float2 *__restrict__ partial, const float *__restrict__ off, Dims dm,
+                    float sl2, int nsplit, int *err) {
+  using C = SCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const int R = dm.G * dm.B;
+  const int W = R / 128;
+  const int nsoft = W * 128;
+  uint8_t *base = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t *sQ = base;
+  uint8_t *sK = sQ + (size_t)W * C::TILE;
+  SBars *bar = reinterpret_cast<SBars *>(sK + (size_t)C::KS * C::TILE);
+  float *sNegOff = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bar) +
+                                             sizeof(uint64_t) * 32);  // [R]
+  float *red = sNegOff + R;                                           // [2][kMaxW][128]
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(red + 2 * kMaxW * 128);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pw = 4 * W;  // producer warp; the MMA warp is pw + 1
+  const int bh = blockIdx.y, b = bh / dm.hkv, h = bh % dm.hkv;
+  const int split = blockIdx.x;
+  const int ntile = (dm.n + kKT - 1) / kKT;
+  const int t0 = (int)((long long)split * ntile / nsplit);
+  const int nt = (int)((long long)(split + 1) * ntile / nsplit) - t0;
+
+  if (tid == 0) {
+    mbar_init(&bar->q_full, 1);
+    for (int s = 0; s < C::KS; ++s) {
+      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->k_empty[s], 1);
+    }
+    for (int w = 0; w < W; ++w) {
+      mbar_init(&bar->s_full[w], 1);
+      mbar_init(&bar->s_free[w], 4);
+    }
+    mbar_init(&bar->mma_done, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == pw + 1) {
+    tmem_alloc(s_tmem, W == 1 ? 128 : W == 2 ? 256 : 512);
+    tmem_relinquish();
+  }
+  if (PASS == 1)
+    for (int r = tid; r < R; r += blockDim.x) sNegOff[r] = -off[(size_t)bh * R + r];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *s_tmem;
+
+  if (warp == pw && lane == 0) {
+    // ------------------------------------------------------- TMA loads
+    bool q_issued = false;
+    int issued = 0;
+    if (nt > 0) {
+      prefetch_map(&tmQ);
+      prefetch_map(&tmK);
+      // probe row r = gl * B + i is row n - B + i of query head h G + gl;
+      // 128-row tile r / 128 of the Q array, each tile stored as H boxes.
+      mbar_expect_tx(&bar->q_full, (uint32_t)W * C::TILE);
+      for (int gl = 0; gl < dm.G; ++gl) {
+        const int r0 = gl * dm.B;
+        const int grow = (b * dm.hq + h * dm.G + gl) * dm.n + dm.n - dm.B;
+        for (int hh = 0; hh < C::H; ++hh)
+          tma_load_2d(sQ + (size_t)(r0 / 128) * C::TILE + hh * C::HALF + (r0 % 128) * 128, &tmQ,
+                      &bar->q_full, hh * 64, grow);
+      }
+      q_issued = true;
+      for (int it = 0; it < nt; ++it) {
+        const int s = it % C::KS, u = it / C::KS;
+        if (u > 0 && !mbar_wait(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 51)) break;
+        mbar_expect_tx(&bar->k_full[s], C::TILE);
+        for (int hh = 0; hh < C::H; ++hh)
+          tma_load_2d(sK + (size_t)s * C::TILE + hh * C::HALF, &tmK, &bar->k_full[s], hh * 64,
+                      bh * dm.n + (t0 + it) * kKT);
+        issued = it + 1;
+      }
+    }
+    // drain: every copy started here lands before the CTA exits
+    int never = 0;
+    if (q_issued) mbar_wait(&bar->q_full, 0, &never, nullptr);
+    for (int t = issued > C::KS ? issued - C::KS : 0; t < issued; ++t)
+      mbar_wait(&bar->k_full[t % C::KS], (t / C::KS) & 1, &never, nullptr);
+  } else if (warp == pw + 1 && lane == 0) {
+    // -------------------------------------------------------- MMA issue
+    // Both operands K-major with the 128-byte swizzle; a k-step of 16 moves
+    // 32 bytes inside a 64-column box, every 4 steps to the next box.
+    constexpr uint32_t kId = idesc_bf16(128, kKT, false);
+    const uint32_t hi = sw128_desc_hi(1024);
+    const uint32_t lo_q = sw128_desc_lo(smem_u32(sQ), 16);
+    const uint32_t lo_k = sw128_desc_lo(smem_u32(sK), 16);
+    if (nt > 0 && mbar_wait(&bar->q_full, 0, s_abort, err, 52)) {
+      tc_fence_after();
+      int ks = 0, kph = 0;
+      for (int it = 0; it < nt; ++it) {
+        if (!mbar_wait(&bar->k_full[ks], kph, s_abort, err, 53)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int w = 0; w < W; ++w) {
+          if (it > 0 && !mbar_wait(&bar->s_free[w], (it - 1) & 1, s_abort, err, 54)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t lq = lo_q + w * (C::TILE >> 4);
+          const uint32_t lk = lo_k + ks * (C::TILE >> 4);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t step = ((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4;
+            const uint64_t dq = desc_words(lq + step, hi), dk = desc_words(lk + step, hi);
+            if (PASS == 0)
+              mma_ss(tbase + w * 128, dq, dk, kId, kk > 0);  // rows x keys
+            else
+              mma_ss(tbase + w * 128, dk, dq, kId, kk > 0);  // keys x rows
+          }
+          mma_commit(&bar->s_full[w]);
+        }
+        if (!ok) break;
+        mma_commit(&bar->k_empty[ks]);
+        if (++ks == C::KS) ks = 0, kph ^= 1;
+      }
+    }
+    // drain: every MMA issued here completes before TMEM is released
+    mma_commit(&bar->mma_done);
+    int never = 0;
+    mbar_wait(&bar->mma_done, 0, &never, nullptr);
+  } else if (warp < pw) {
+    // ------------------------------------------------------- row groups
+    const int w = warp >> 2, quarter = warp & 3;
+    const int lrow = quarter * 32 + lane;  // this thread's TMEM lane
+    const uint32_t tS = tbase + w * 128 + ((uint32_t)(quarter * 32) << 16);
+    const float2 sl2x2 = make_float2(sl2, sl2);
+    // pass 1: this lane is probe row r at sequence position pos
+    const int r = w * 128 + lrow;
+    const int pos = dm.n - dm.B + r % dm.B;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int it = 0; it < nt; ++it) {
+      const int key0 = (t0 + it) * kKT;
+      const bool edge = key0 + kKT > dm.n - dm.B;  // causal mask or tail inside
+      if (ok && !mbar_wait_warp(&bar->s_full[w], it & 1, s_abort, err, 55)) ok = false;
+      float part = 0.f;
+      if (ok) {
+        tc_fence_after();
+        uint32_t va[32], vb[32];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          tmem_ld32(tS + hf * 64, va);
+          tmem_ld32(tS + hf * 64 + 32, vb);
+          tmem_wait_ld();
+          if (hf == 1) {  // the slice is in registers: the next tile may overwrite it
+            tc_fence_before();
+            warp_arrive(&bar->s_free[w], lane);
+          }
+          if (PASS == 0) {
+            // ---- running max and sum of this row over 64 keys
+            float v[64];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(va[c]), v[32 + c] = __uint_as_float(vb[c]);
+            if (edge) {
+              const int kb = key0 + hf * 64;
+#pragma unroll
+              for (int c = 0; c < 64; ++c)
+                if (kb + c > pos || kb + c >= dm.n) v[c] = -INFINITY;
+            }
+            float c0 = v[0], c1 = v[1], c2 = v[2], c3 = v[3];
+#pragma unroll
+            for (int c = 4; c < 64; c += 4)
+              c0 = fmaxf(c0, v[c]), c1 = fmaxf(c1, v[c + 1]), c2 = fmaxf(c2, v[c + 2]),
+              c3 = fmaxf(c3, v[c + 3]);
+            const float mn = fmaxf(m, fmaxf(fmaxf(c0, c1), fmaxf(c2, c3)) * sl2);
+            if (mn > m) {
+              l *= ex2_approx(m - mn);
+              m = mn;
+            }
+            const float mu = m == -INFINITY ? 0.f : m;  // nothing visible yet
+            const float2 nm = make_float2(-mu, -mu);
+            float2 a[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) a[x] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              const float2 t = __ffma2_rn(make_float2(v[c], v[c + 1]), sl2x2, nm);
+              a[(c >> 1) & 3] =
+                  __fadd2_rn(a[(c >> 1) & 3], make_float2(ex2_approx(t.x), ex2_approx(t.y)));
+            }
+            const float2 s = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+            l += s.x + s.y;
+          } else {
+            // ---- this key's probabilities over 64 probe rows
+            const int key = key0 + lrow;
+            const int rb = w * 128 + hf * 64;
+            float2 a[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) a[x] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+              const float4 no = *reinterpret_cast<const float4 *>(&sNegOff[rb + c]);
+              const uint32_t *src = c < 32 ? &va[c] : &vb[c - 32];
+              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+                                     sl2x2, make_float2(no.x, no.y));
+              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+                                     sl2x2, make_float2(no.z, no.w));
+              if (edge) {
+                const int p0 = dm.n - dm.B;
+                if (key > p0 + (rb + c) % dm.B) t0.x = -INFINITY;
+                if (key > p0 + (rb + c + 1) % dm.B) t0.y = -INFINITY;
+                if (key > p0 + (rb + c + 2) % dm.B) t1.x = -INFINITY;
+                if (key > p0 + (rb + c + 3) % dm.B) t1.y = -INFINITY;
+              }
+              a[(c >> 2) & 1] =
+                  __fadd2_rn(a[(c >> 2) & 1], make_float2(ex2_approx(t0.x), ex2_approx(t0.y)));
+              a[2 + ((c >> 2) & 1)] =
+                  __fadd2_rn(a[2 + ((c >> 2) & 1)], make_float2(ex2_approx(t1.x), ex2_approx(t1.y)));
+            }
+            const float2 s = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+            part += s.x + s.y;
+          }
+        }
+      }
+      if (PASS == 1) {
+        // The row groups' partial sums of each key, added in group order.
+        // Every row-group thread takes this barrier once per tile, also after
+        // a failed wait, so none is left waiting.
+        float *rb = red + (it & 1) * kMaxW * 128;
+        rb[w * 128 + lrow] = part;
+        softmax_bar(nsoft);
+        if (w == 0) {
+          float s = rb[lrow];
+          for (int x = 1; x < W; ++x) s += rb[x * 128 + lrow];
+          const int key = key0 + lrow;
+          if (ok && key < dm.n) imp[(size_t)bh * dm.n + key] = s / (float)R;
+        }
+      }
+    }
+    if (PASS == 0 && ok && nt > 0)
+      partial[((size_t)bh * nsplit + split) * R + r] = make_float2(m, l);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == pw + 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tbase, W == 1 ? 128 : W == 2 ? 256 : 512);
+  }
+}
+
+// Per row: M = max over CTAs of m, L = sum of l 2^(m - M); off = M + log2 L.
+__global__ void score_tc_combine(const float2 *__restrict__ partial, float *__restrict__ off,
+                                 int R, int nsplit, int total) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  const int bh = i / R, r = i % R;
+  const float2 *p = partial + (size_t)bh * nsplit * R + r;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[(size_t)s * R].x);
+  float L = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const float2 v = p[(size_t)s * R];
+    if (v.x != -INFINITY) L += v.y * exp2f(v.x - M);
+  }
+  off[i] = M + log2f(L);
+}
+
+int sm_count() {
+  int dev = 0, c = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return c;
+}
+
+// CTAs per (batch, KV head): one wave over the SMs, at most one per tile.
+int tc_splits(const Dims &dm) {
+  const int bh = dm.b * dm.hkv;
+  const int ntile = (dm.n + kKT - 1) / kKT;
+  int s = sm_count() / bh;
+  if (s > ntile) s = ntile;
+  return s < 1 ? 1 : s;
+}
+
+template <int D>
+cudaError_t run_tc(const Dims &dm, const void *q, const void *k, float *imp, float sigma,
+                   void *ws, int *err, cudaStream_t st) {
+  const int R = dm.G * dm.B;
+  const int nsplit = tc_splits(dm);
+  const int bh = dm.b * dm.hkv;
+  CUtensorMap mq, mk;
+  if (!make_tile_map(&mq, q, (uint64_t)dm.b * dm.hq * dm.n, D, dm.B) ||
+      !make_tile_map(&mk, k, (uint64_t)dm.b * dm.hkv * dm.n, D, kKT))
+    return cudaErrorInvalidValue;
+  const size_t smem = SCfg<D>::smem(R);
+  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D, 0>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(score_tc_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+  if (e != cudaSuccess) return e;
+  float2 *partial = reinterpret_cast<float2 *>(ws);
+  float *off = reinterpret_cast<float *>(partial + (size_t)bh * nsplit * R);
+  const dim3 grid(nsplit, bh);
+  const int threads = R + 64;
+  const float sl2 = sigma * kLog2e;
+  score_tc_kernel<D, 0><<<grid, threads, smem, st>>>(mq, mk, imp, partial, off, dm, sl2, nsplit,
+                                                     err);
+  const int total = bh * R;
+  score_tc_combine<<<(total + 255) / 256, 256, 0, st>>>(partial, off, R, nsplit, total);
+  score_tc_kernel<D, 1><<<grid, threads, smem, st>>>(mq, mk, imp, partial, off, dm, sl2, nsplit,
+                                                     err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool score_tc_supported(const Dims &dm) {
+  const int R = dm.G * dm.B;
+  if (R % 128 != 0 || R > 128 * kMaxW || (dm.B != 64 && dm.B != 128)) return false;
+  if (dm.d == 64) return SCfg<64>::smem(R) <= 227 * 1024;
+  if (dm.d == 128) return SCfg<128>::smem(R) <= 227 * 1024;
+  return false;
+}
+
+size_t score_tc_ws_bytes(const Dims &dm) {
+  const size_t R = (size_t)dm.G * dm.B, bh = (size_t)dm.b * dm.hkv;
+  return bh * tc_splits(dm) * R * sizeof(float2) + bh * R * sizeof(float);
+}
+
+cudaError_t launch_score_tc(const Dims &dm, const void *q, const void *k, float *imp,
+                            float sigma, void *ws, int *err, cudaStream_t st) {
+  if (dm.d == 64) return run_tc<64>(dm, q, k, imp, sigma, ws, err, st);
+  return run_tc<128>(dm, q, k, imp, sigma, ws, err, st);
+}
+
+}  // namespace pbs

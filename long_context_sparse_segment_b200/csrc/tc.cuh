@@ -7,6 +7,12 @@
 #include "common.cuh"
 
 namespace pbs {
+
+// Host: a 2-D tensor map over `rows` rows of d bf16 values, boxes of 64
+// columns (128 bytes, the 128-byte swizzle) by `box_rows` rows. False when
+// the driver's encoder is unavailable or rejects the arguments.
+bool make_tile_map(CUtensorMap *map, const void *ptr, uint64_t rows, int d, int box_rows);
+
 namespace tc {
 
 // Bounded waits: a wait that has not completed after this long records

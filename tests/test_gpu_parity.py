@@ -218,3 +218,36 @@ def test_tensor_core_and_warp_mma_forwards_agree(name, dev, monkeypatch):
     assert_outputs_close(f64(o_mma), ref, "warp mma")
     np.testing.assert_allclose(f64(lse_tc), f64(lse_mma), atol=1e-3)
     assert pbs.device_status() == 0
+
+
+SCORE_SHAPES = {
+    # (batch, hq, hkv, n, d, B): G*B = 512, 256, 384 and 128 take the tcgen05
+    # kernel, G*B = 64 the warp-MMA kernel
+    "r512_d128": (1, 8, 2, 2048, 128, 128),
+    "r256_b2": (2, 4, 2, 1280, 128, 128),
+    "r384": (1, 6, 2, 1536, 128, 128),
+    "r512_d64": (1, 4, 1, 1024, 64, 128),
+    # B = 64 probe rows, n % 128 == 64: the last key tile is half past the end
+    "r128_b64_tail": (1, 4, 2, 1088, 128, 64),
+    "r64_mma": (1, 4, 4, 1024, 128, 64),
+}
+
+
+@pytest.mark.parametrize("name", list(SCORE_SHAPES))
+def test_score_kernels_against_oracle(name, dev, monkeypatch):
+    """Both scoring kernels (tcgen05 and warp-MMA) against the oracle's
+    importance, and against each other."""
+    b, hq, hkv, n, d, B = SCORE_SHAPES[name]
+    w = Workload(name, b, hq, hkv, n, d, B, n, "threshold", 0.9, "uniform", 0.05, seed=3)
+    (q, k, _), (qd, kd, _) = inputs(w, dev)
+    want = orc.score(f64(q), f64(k), B)
+    imp_tc = pbs.score(qd, kd, B)
+    monkeypatch.setenv("PBS_SCORE", "mma")
+    imp_mma = pbs.score(qd, kd, B)
+    monkeypatch.delenv("PBS_SCORE")
+    torch.cuda.synchronize()
+    assert pbs.device_status() == 0
+    assert_importance_close(f64(imp_tc), want)
+    assert_importance_close(f64(imp_mma), want)
+    # the two kernels sum in different orders: agreement to fp32 rounding
+    np.testing.assert_allclose(f64(imp_tc), f64(imp_mma), rtol=1e-4, atol=0)
