@@ -12,24 +12,31 @@
 // The two passes use opposite operand roles so that every reduction is
 // local to a thread, with no shuffles:
 //   pass 1: D = Q_w K_t^T, Q rows on the MMA's M side: the TMEM lane is a
-//           probe row, its columns are keys. Each thread keeps its row's
+//           probe row, its columns are keys. Each thread keeps its rows'
 //           running max and sum of exp2 -> partial (m, l) per (row, CTA).
 //   combine: per row, M = max m, L = sum l 2^(m - M); off = M + log2 L.
 //   pass 2: D = K_t Q_w^T, keys on the M side: the TMEM lane is a key, its
 //           columns are probe rows. p = 2^(s - off_r) summed over the
-//           thread's columns; the R/128 row groups' partial sums of a key
-//           are added in a fixed order -> imp = sum / R. Deterministic, no
+//           thread's columns; the warpgroups' partial sums of a key are
+//           added in a fixed order -> imp = sum / R. Deterministic, no
 //           atomics.
 // Logits are in log2 units: s = (q . k) sigma log2(e).
 //
-// Roles (R/128 = W row groups; 128 W + 64 threads):
-//   warps 0 .. 4W-1   one warpgroup per 128-column TMEM slice w (probe rows
-//                     128w .. 128w+127); thread = TMEM lane;
-//   warp 4W, lane 0   TMA: the probe rows once, then K tiles into a ring;
-//   warp 4W+1, lane 0 tcgen05.mma issue: per K tile, one 128 x 128 x d
-//                     product per slice, each released as soon as its
-//                     warpgroup has read the slice into registers.
-// Every mbarrier wait is bounded (PBS_ERR_TIMEOUT, the CTA drains and exits).
+// TMEM holds one 128 x 128 fp32 slice per 128 probe rows (W = R/128 slices,
+// all 512 columns at R = 512). Roles:
+//   warps 0 .. 4W-1    warpgroup w owns slice w; a thread is a TMEM lane. It
+//                      reads the slice into registers in two 64-column
+//                      halves and releases it once the second half is read,
+//                      so the tensor core refills it with the next tile
+//                      while the second half is worked on;
+//   warp 4W, lane 0    TMA: the probe rows once, then K tiles into a ring;
+//   warp 4W+1, lane 0  tcgen05.mma issue: per K tile and slice one
+//                      128 x 128 x d product, issued once the slice is free.
+// (Measured on B200: this beats releasing 64-column halves separately with
+// 128 x 64 products, and two warpgroups that each hold a whole slice.)
+// 2^x is split between the MUFU unit and an FMA-pipe polynomial, which
+// together bound both passes. Every mbarrier wait is bounded
+// (PBS_ERR_TIMEOUT, the CTA drains and exits).
 #include <math.h>
 
 #include "common.cuh"
@@ -45,13 +52,14 @@ using namespace tc;
 constexpr int kKT = 128;   // keys per tile
 constexpr int kMaxW = 4;   // R <= 512
 constexpr int kMaxKS = 4;  // K ring depth (upper bound)
+constexpr int kMaxThreads = kMaxW * 128 + 64;
 
 template <int D>
 struct SCfg {
-  static constexpr int H = D / 64;                         // 64-column boxes per row
-  static constexpr uint32_t TILE = 128u * D * 2;           // bytes of one 128-row tile
-  static constexpr uint32_t HALF = 128u * 128;             // bytes of one 64-column box
-  static constexpr int KS = D == 128 ? 2 : 4;              // K ring depth
+  static constexpr int H = D / 64;                // 64-column boxes per row
+  static constexpr uint32_t TILE = 128u * D * 2;  // bytes of one 128-row tile
+  static constexpr uint32_t HALF = 128u * 128;    // bytes of one 64-column box
+  static constexpr int KS = D == 128 ? 2 : 4;     // K ring depth
   static size_t smem(int R) {
     return 1024 + (size_t)(R / 128) * TILE + (size_t)KS * TILE + sizeof(uint64_t) * 32 +
            (size_t)R * 4 + 2 * kMaxW * 128 * 4 + 16;
@@ -63,12 +71,28 @@ struct SBars {
 };
 static_assert(sizeof(SBars) <= sizeof(uint64_t) * 32, "barrier block");
 
-__device__ __forceinline__ void softmax_bar(int nthreads) {
+// 2^t for a pair: pairs 3, 6 and 7 of every 8 (37.5%) go to the FMA pipe,
+// the rest to the MUFU unit, which alone would bound both passes. The
+// quartic keeps the sums within a few 1e-6 of exact.
+__device__ __forceinline__ float2 exp2_split(float2 t, int pair) {
+  const int k = pair & 7;
+  if (k == 3 || k == 6 || k == 7) return exp2_poly4x2(t);
+  return make_float2(ex2_approx(t.x), ex2_approx(t.y));
+}
+
+__device__ __forceinline__ void rows_bar(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
+// Half a slice (64 TMEM columns) of this thread's lane into registers.
+__device__ __forceinline__ void load_half(uint32_t taddr, uint32_t (&v)[64]) {
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+  tmem_wait_ld();
+}
+
 template <int D, int PASS>
-__global__ void __launch_bounds__(kMaxW * 128 + 64, 1)
+__global__ void __launch_bounds__(kMaxThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, float *__restrict__ imp,
                     float2 *__restrict__ partial, const float *__restrict__ off, Dims dm,
@@ -77,7 +101,6 @@ __global__ void __launch_bounds__(kMaxW * 128 + 64, 1)
   extern __shared__ uint8_t smem_raw[];
   const int R = dm.G * dm.B;
   const int W = R / 128;
-  const int nsoft = W * 128;
   uint8_t *base = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t *sQ = base;
@@ -96,6 +119,7 @@ __global__ void __launch_bounds__(kMaxW * 128 + 64, 1)
   const int ntile = (dm.n + kKT - 1) / kKT;
   const int t0 = (int)((long long)split * ntile / nsplit);
   const int nt = (int)((long long)(split + 1) * ntile / nsplit) - t0;
+  const uint32_t tcols = W == 1 ? 128 : W == 2 ? 256 : 512;
 
   if (tid == 0) {
     mbar_init(&bar->q_full, 1);
@@ -105,14 +129,14 @@ __global__ void __launch_bounds__(kMaxW * 128 + 64, 1)
     }
     for (int w = 0; w < W; ++w) {
       mbar_init(&bar->s_full[w], 1);
-      mbar_init(&bar->s_free[w], 4);
+      mbar_init(&bar->s_free[w], 4);  // the four warps of warpgroup w
     }
     mbar_init(&bar->mma_done, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
   if (warp == pw + 1) {
-    tmem_alloc(s_tmem, W == 1 ? 128 : W == 2 ? 256 : 512);
+    tmem_alloc(s_tmem, tcols);
     tmem_relinquish();
   }
   if (PASS == 1)
@@ -166,26 +190,25 @@ __global__ void __launch_bounds__(kMaxW * 128 + 64, 1)
     if (nt > 0 && mbar_wait(&bar->q_full, 0, s_abort, err, 52)) {
       tc_fence_after();
       int ks = 0, kph = 0;
-      for (int it = 0; it < nt; ++it) {
+      bool ok = true;
+      for (int it = 0; it < nt && ok; ++it) {
         if (!mbar_wait(&bar->k_full[ks], kph, s_abort, err, 53)) break;
         tc_fence_after();
-        bool ok = true;
         for (int w = 0; w < W; ++w) {
           if (it > 0 && !mbar_wait(&bar->s_free[w], (it - 1) & 1, s_abort, err, 54)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t lq = lo_q + w * (C::TILE >> 4);
-          const uint32_t lk = lo_k + ks * (C::TILE >> 4);
+          // pass 1: A = Q rows of slice w, B = the K tile (rows x keys);
+          // pass 2: A = the K tile, B = Q rows of slice w (keys x rows)
+          const uint32_t lq = lo_q + w * (C::TILE >> 4), lk = lo_k + ks * (C::TILE >> 4);
+          const uint32_t la = PASS == 0 ? lq : lk, lb = PASS == 0 ? lk : lq;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t step = ((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4;
-            const uint64_t dq = desc_words(lq + step, hi), dk = desc_words(lk + step, hi);
-            if (PASS == 0)
-              mma_ss(tbase + w * 128, dq, dk, kId, kk > 0);  // rows x keys
-            else
-              mma_ss(tbase + w * 128, dk, dq, kId, kk > 0);  // keys x rows
+            mma_ss(tbase + w * 128, desc_words(la + step, hi), desc_words(lb + step, hi), kId,
+                   kk > 0);
           }
           mma_commit(&bar->s_full[w]);
         }
@@ -212,93 +235,91 @@ __global__ void __launch_bounds__(kMaxW * 128 + 64, 1)
     for (int it = 0; it < nt; ++it) {
       const int key0 = (t0 + it) * kKT;
       const bool edge = key0 + kKT > dm.n - dm.B;  // causal mask or tail inside
-      if (ok && !mbar_wait_warp(&bar->s_full[w], it & 1, s_abort, err, 55)) ok = false;
       float part = 0.f;
-      if (ok) {
-        tc_fence_after();
-        uint32_t va[32], vb[32];
+      if (ok && !mbar_wait_warp(&bar->s_full[w], it & 1, s_abort, err, 55)) ok = false;
+      if (ok) tc_fence_after();
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        if (!ok) break;
+        uint32_t v[64];
+        load_half(tS + hf * 64, v);
+        if (hf == 1) {  // the slice is in registers: the next tile may overwrite it
+          tc_fence_before();
+          warp_arrive(&bar->s_free[w], lane);
+        }
+        if (PASS == 0) {
+          // ---- probe row r over keys key0 + 64 hf .. + 63
+          if (edge) {
+            const int lim = pos - key0 - hf * 64;  // last visible column
+            const int end = dm.n - key0 - hf * 64;  // first column past n
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          tmem_ld32(tS + hf * 64, va);
-          tmem_ld32(tS + hf * 64 + 32, vb);
-          tmem_wait_ld();
-          if (hf == 1) {  // the slice is in registers: the next tile may overwrite it
-            tc_fence_before();
-            warp_arrive(&bar->s_free[w], lane);
+            for (int c = 0; c < 64; ++c)
+              if (c > lim || c >= end) v[c] = 0xff800000u;  // -inf
           }
-          if (PASS == 0) {
-            // ---- running max and sum of this row over 64 keys
-            float v[64];
+          float c0 = __uint_as_float(v[0]), c1 = __uint_as_float(v[1]);
+          float c2 = __uint_as_float(v[2]), c3 = __uint_as_float(v[3]);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(va[c]), v[32 + c] = __uint_as_float(vb[c]);
-            if (edge) {
-              const int kb = key0 + hf * 64;
-#pragma unroll
-              for (int c = 0; c < 64; ++c)
-                if (kb + c > pos || kb + c >= dm.n) v[c] = -INFINITY;
-            }
-            float c0 = v[0], c1 = v[1], c2 = v[2], c3 = v[3];
-#pragma unroll
-            for (int c = 4; c < 64; c += 4)
-              c0 = fmaxf(c0, v[c]), c1 = fmaxf(c1, v[c + 1]), c2 = fmaxf(c2, v[c + 2]),
-              c3 = fmaxf(c3, v[c + 3]);
-            const float mn = fmaxf(m, fmaxf(fmaxf(c0, c1), fmaxf(c2, c3)) * sl2);
-            if (mn > m) {
-              l *= ex2_approx(m - mn);
-              m = mn;
-            }
-            const float mu = m == -INFINITY ? 0.f : m;  // nothing visible yet
-            const float2 nm = make_float2(-mu, -mu);
-            float2 a[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) a[x] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-              const float2 t = __ffma2_rn(make_float2(v[c], v[c + 1]), sl2x2, nm);
-              a[(c >> 1) & 3] =
-                  __fadd2_rn(a[(c >> 1) & 3], make_float2(ex2_approx(t.x), ex2_approx(t.y)));
-            }
-            const float2 s = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
-            l += s.x + s.y;
-          } else {
-            // ---- this key's probabilities over 64 probe rows
-            const int key = key0 + lrow;
-            const int rb = w * 128 + hf * 64;
-            float2 a[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) a[x] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int c = 0; c < 64; c += 4) {
-              const float4 no = *reinterpret_cast<const float4 *>(&sNegOff[rb + c]);
-              const uint32_t *src = c < 32 ? &va[c] : &vb[c - 32];
-              float2 t0 = __ffma2_rn(make_float2(__uint_as_float(src[0]), __uint_as_float(src[1])),
-                                     sl2x2, make_float2(no.x, no.y));
-              float2 t1 = __ffma2_rn(make_float2(__uint_as_float(src[2]), __uint_as_float(src[3])),
-                                     sl2x2, make_float2(no.z, no.w));
-              if (edge) {
-                const int p0 = dm.n - dm.B;
-                if (key > p0 + (rb + c) % dm.B) t0.x = -INFINITY;
-                if (key > p0 + (rb + c + 1) % dm.B) t0.y = -INFINITY;
-                if (key > p0 + (rb + c + 2) % dm.B) t1.x = -INFINITY;
-                if (key > p0 + (rb + c + 3) % dm.B) t1.y = -INFINITY;
-              }
-              a[(c >> 2) & 1] =
-                  __fadd2_rn(a[(c >> 2) & 1], make_float2(ex2_approx(t0.x), ex2_approx(t0.y)));
-              a[2 + ((c >> 2) & 1)] =
-                  __fadd2_rn(a[2 + ((c >> 2) & 1)], make_float2(ex2_approx(t1.x), ex2_approx(t1.y)));
-            }
-            const float2 s = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
-            part += s.x + s.y;
+          for (int c = 4; c < 64; c += 4) {
+            c0 = fmaxf(c0, __uint_as_float(v[c]));
+            c1 = fmaxf(c1, __uint_as_float(v[c + 1]));
+            c2 = fmaxf(c2, __uint_as_float(v[c + 2]));
+            c3 = fmaxf(c3, __uint_as_float(v[c + 3]));
           }
+          const float mn = fmaxf(m, fmaxf(fmaxf(c0, c1), fmaxf(c2, c3)) * sl2);
+          if (mn > m) {
+            l *= ex2_approx(m - mn);
+            m = mn;
+          }
+          const float mu = m == -INFINITY ? 0.f : m;  // nothing visible yet
+          const float2 nm = make_float2(-mu, -mu);
+          float2 a[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) a[x] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float2 t = __ffma2_rn(
+                make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sl2x2, nm);
+            a[(c >> 1) & 3] = __fadd2_rn(a[(c >> 1) & 3], exp2_split(t, c >> 1));
+          }
+          const float2 s = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+          l += s.x + s.y;
+        } else {
+          // ---- key key0 + lrow over probe rows 128 w + 64 hf .. + 63
+          const int rb = w * 128 + hf * 64;
+          if (edge) {
+            // probe row q (position n - B + q mod B) sees the key only if
+            // q mod B >= key - (n - B); keys past n are seen by none
+            const int lim = key0 + lrow - (dm.n - dm.B);
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (((rb + c) & (dm.B - 1)) < lim) v[c] = 0xff800000u;  // -inf
+          }
+          float2 a[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) a[x] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            const float4 no = *reinterpret_cast<const float4 *>(&sNegOff[rb + c]);
+            const float2 ta = __ffma2_rn(
+                make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sl2x2,
+                make_float2(no.x, no.y));
+            const float2 tb = __ffma2_rn(
+                make_float2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3])), sl2x2,
+                make_float2(no.z, no.w));
+            a[(c >> 2) & 1] = __fadd2_rn(a[(c >> 2) & 1], exp2_split(ta, c >> 1));
+            a[2 + ((c >> 2) & 1)] = __fadd2_rn(a[2 + ((c >> 2) & 1)], exp2_split(tb, (c >> 1) + 1));
+          }
+          const float2 s = __fadd2_rn(__fadd2_rn(a[0], a[1]), __fadd2_rn(a[2], a[3]));
+          part += s.x + s.y;
         }
       }
       if (PASS == 1) {
-        // The row groups' partial sums of each key, added in group order.
+        // The warpgroups' partial sums of each key, added in slice order.
         // Every row-group thread takes this barrier once per tile, also after
         // a failed wait, so none is left waiting.
         float *rb = red + (it & 1) * kMaxW * 128;
         rb[w * 128 + lrow] = part;
-        softmax_bar(nsoft);
+        rows_bar(W * 128);
         if (w == 0) {
           float s = rb[lrow];
           for (int x = 1; x < W; ++x) s += rb[x * 128 + lrow];
@@ -315,7 +336,7 @@ __global__ void __launch_bounds__(kMaxW * 128 + 64, 1)
   if (warp == pw + 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tbase, W == 1 ? 128 : W == 2 ? 256 : 512);
+    tmem_dealloc(tbase, tcols);
   }
 }
 
