@@ -255,21 +255,31 @@ cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const
 
 namespace pbs {
 
-// The tensor-core (tcgen05) kernel serves B = 128 with d = 64 or 128; the
-// warp-MMA kernel serves B = 64. PBS_FORWARD=mma selects the warp-MMA kernel
-// for every shape (a diagnostic switch for comparing the two).
-// PBS_FAULT_INJECT=timeout makes the tcgen05 kernel skip its first K' load,
-// so that its bounded waits run out and it reports PBS_ERR_TIMEOUT (used by
-// the failure-detection test).
+// The tensor-core (tcgen05) kernels serve B = 128 with d = 64 or 128: by
+// default the one with two query tiles per CTA, PBS_FORWARD=tc1 the one with
+// one tile per CTA; the warp-MMA kernel serves B = 64, and every shape under
+// PBS_FORWARD=mma (diagnostic switches for comparing the kernels). The
+// two-tile kernel refuses to launch (cudaErrorInvalidConfiguration) unless
+// it was compiled at the register count its register split assumes; the
+// one-tile kernel then runs instead.
+// PBS_FAULT_INJECT=timeout makes the tcgen05 kernels skip their first K'
+// load, so that their bounded waits run out and they report
+// PBS_ERR_TIMEOUT (used by the failure-detection test).
 cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const void *vp,
                         const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                         const int32_t *cnt, void *out, float *lse, float sigma, int *err,
                         cudaStream_t st) {
   const char *fwd = getenv("PBS_FORWARD");
   const bool force_mma = fwd && strcmp(fwd, "mma") == 0;
+  const bool force_tc1 = fwd && strcmp(fwd, "tc1") == 0;
   if (attn_tc_supported(dm) && !force_mma) {
     const char *fi = getenv("PBS_FAULT_INJECT");
     const int fault = (fi && strcmp(fi, "timeout") == 0) ? 1 : 0;
+    if (!force_tc1) {
+      const cudaError_t e =
+          launch_attn_tc2(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, st);
+      if (e != cudaErrorInvalidConfiguration) return e;
+    }
     return launch_attn_tc(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, st);
   }
   return launch_attn_mma(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, st);

@@ -57,6 +57,12 @@ cudaError_t launch_attn_tc(const Dims &dm, const void *q, const void *kp, const 
                            const int32_t *cnt, void *out, float *lse, float sigma, int *err,
                            int fault, cudaStream_t st);
 
+// the same forward with two query tiles per CTA (tcgen05; B = 128, d in {64, 128})
+cudaError_t launch_attn_tc2(const Dims &dm, const void *q, const void *kp, const void *vp,
+                            const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
+                            const int32_t *cnt, void *out, float *lse, float sigma, int *err,
+                            int fault, cudaStream_t st);
+
 // the same forward on the legacy warp-MMA path
 cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,

@@ -39,6 +39,10 @@ CASES = {
     # S = B: one block per segment
     "s_eq_b": Workload("s_eq_b", 1, 4, 2, 1024, 128, 128, 128, "threshold", 0.9,
                        "uniform", 0.05),
+    # an odd number of (head, query block) items: the last CTA of the
+    # two-tile forward has one tile
+    "odd_items": Workload("odd_items", 1, 3, 1, 1152, 128, 128, 384, "topk_frac", 0.4,
+                          "uniform", 0.05),
     # S = N: one segment, every block forced
     "s_eq_n": Workload("s_eq_n", 1, 2, 1, 1024, 64, 64, 1024, "threshold", 0.5,
                        "uniform", 0.05),
@@ -197,7 +201,7 @@ def test_device_status_is_clean(dev):
     assert pbs.device_status() == 0
 
 
-@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128"])
+@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128", "odd_items"])
 def test_tensor_core_and_warp_mma_forwards_agree(name, dev, monkeypatch):
     """The tcgen05 forward and the warp-MMA forward on the same lists, each
     against the oracle."""
@@ -251,3 +255,33 @@ def test_score_kernels_against_oracle(name, dev, monkeypatch):
     assert_importance_close(f64(imp_mma), want)
     # the two kernels sum in different orders: agreement to fp32 rounding
     np.testing.assert_allclose(f64(imp_tc), f64(imp_mma), rtol=1e-4, atol=0)
+
+
+@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128", "odd_items", "s_eq_b"])
+@pytest.mark.parametrize("permute_q", [False, True])
+def test_two_tile_and_one_tile_forwards_agree(name, permute_q, dev, monkeypatch):
+    """The two-tile tcgen05 forward (the default) and the one-tile one on the
+    same lists: both against the oracle, and equal to bf16 rounding."""
+    w = CASES[name]
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    imp = pbs.score(qd, kd, B)
+    perm = pbs.permute(imp, kd, vd, B, S, q=qd if permute_q else None, hq=w.hq)
+    q_used = perm["q_perm"] if permute_q else qd
+    qpos = perm["kpos"] if permute_q else None
+    idx, cnt, _ = pbs.select_blocks(q_used, perm["k_perm"], perm["kbar_sum"], B, S, w.mode,
+                                    w.param)
+    args = (q_used, perm["k_perm"], perm["v_perm"], perm["kpos"], qpos, idx, cnt, B, S)
+    o2, lse2 = pbs.attn_fwd(*args, lse=True)
+    monkeypatch.setenv("PBS_FORWARD", "tc1")
+    o1, lse1 = pbs.attn_fwd(*args, lse=True)
+    monkeypatch.delenv("PBS_FORWARD")
+    torch.cuda.synchronize()
+    assert pbs.device_status() == 0
+    qpos64 = None if qpos is None else np.repeat(i64(qpos), w.group, axis=1)
+    ref = orc.attend(f64(q_used), f64(perm["k_perm"]), f64(perm["v_perm"]), i64(perm["kpos"]),
+                     qpos64, i64(idx), i64(cnt), B)
+    assert_outputs_close(f64(o2), ref, "two-tile")
+    assert_outputs_close(f64(o1), ref, "one-tile")
+    assert_outputs_close(f64(o2), f64(o1), "two-tile vs one-tile")
+    np.testing.assert_allclose(f64(lse2), f64(lse1), atol=1e-4)
