@@ -24,8 +24,9 @@
 //   warp 1, one thread   tcgen05.mma issue in the order above;
 //   warps 4-7, 8-11      softmax of tile A, of tile B: one thread per query
 //                        row (TMEM lane), all 128 key columns of a block:
-//                        mask, row max, exp2 (MUFU and an FMA-pipe cubic),
-//                        P to TMEM, row sum; final normalisation and store.
+//                        mask, row max (three-input max), exp2 (MUFU), P to
+//                        TMEM in two halves, row sum; final normalisation
+//                        and store.
 // A softmax thread holds a whole row of S, so the first warpgroup (warps
 // 0-3) gives registers to the other two (setmaxnreg): 128 x 56 + 256 x 224
 // = 64,512, exactly the 384 x 168 the CTA is launched with.
@@ -69,7 +70,7 @@ struct Cfg2 {
 template <int D>
 struct Bars2 {
   uint64_t q_full, k_full[Cfg2<D>::KS], k_empty[Cfg2<D>::KS], v_full[Cfg2<D>::VS],
-      v_empty[Cfg2<D>::VS], s_full[2], p_full[2], o_final[2], mma_done;
+      v_empty[Cfg2<D>::VS], s_full[2], p_full[2][2], o_final[2], mma_done;
 };
 
 template <int D>
@@ -118,6 +119,16 @@ __device__ __forceinline__ int checked_block(const Tile &t, int j, const Dims &d
   return J;
 }
 
+// How many of the 16 exponent pairs of a 32-column chunk go to the FMA-pipe
+// cubic instead of the MUFU unit. Measured on B200 (llama32k, llama128k):
+// 0 is fastest; 4-8 of 16 cost 8-10%. The MUFU unit is not this kernel's
+// limit, and under the power cap the extra FMA-pipe instructions lower the
+// clock more than they save.
+constexpr int kPolyPairs = 0;
+__device__ __forceinline__ constexpr bool poly_pair(int e) {
+  return (e * kPolyPairs) % 16 >= 16 - kPolyPairs;  // spread evenly over the chunk
+}
+
 // Position of block j of tile x (0 = A, 1 = B) in the interleaved stream
 // A0 B0 A1 B1 ... (a list that has ended drops out).
 __device__ __forceinline__ int stream_pos(int x, int j, int cA, int cB) {
@@ -164,7 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bar->s_full[x], 1);
-      mbar_init(&bar->p_full[x], 4);  // the four warps of the tile's softmax
+      mbar_init(&bar->p_full[x][0], 4);  // the four warps of the tile's softmax,
+      mbar_init(&bar->p_full[x][1], 4);  // for keys 0-63 and 64-127 of P
       mbar_init(&bar->o_final[x], 1);
     }
     mbar_init(&bar->mma_done, 1);
@@ -276,15 +288,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // O_x += P_x V': A = P_x from TMEM (bf16 pairs over S_x), B = the V' tile
     // (MN-major); the first block of a tile overwrites O_x
+    // The first half of P (keys 0-63) is consumed while the softmax still
+    // writes the second.
     auto pv = [&](int x, int j) -> bool {
-      if (!mbar_wait(&bar->p_full[x], j & 1, s_abort, err, 33)) return false;
+      if (!mbar_wait(&bar->p_full[x][0], j & 1, s_abort, err, 33)) return false;
       if (!mbar_wait(&bar->v_full[vs], vph, s_abort, err, 34)) return false;
       tc_fence_after();
       const uint32_t lv = lo_v + vs * (C::TILE >> 4);
 #pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
+      for (int kk = 0; kk < kBN / 16; ++kk) {
+        if (kk == kBN / 32) {
+          if (!mbar_wait(&bar->p_full[x][1], j & 1, s_abort, err, 35)) return false;
+          tc_fence_after();
+        }
         mma_ts(tbase + 256 + x * 128, tbase + x * 128 + kk * 8,
                desc_words(lv + kk * (2048 >> 4), hi), kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+      }
       mma_commit(&bar->v_empty[vs]);
       if (++vs == VS) vs = 0, vph ^= 1;
       return true;
@@ -368,15 +387,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c > lim) v[c] = 0xff800000u;
         }
       }
+      // row max: eight chains of three-input max over the 128 columns
       float m8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(v[e]);
 #pragma unroll
-      for (int c = 8; c < kBN; c += 8)
+      for (int c = 8; c + 16 <= kBN; c += 16)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], __uint_as_float(v[c + e]));
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int e = 0; e < 8; ++e)
+          m8[e] = max3f(m8[e], __uint_as_float(v[c + e]), __uint_as_float(v[c + 8 + e]));
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], __uint_as_float(v[kBN - 8 + e]));
+      const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]),
+                             fmaxf(m8[6], m8[7]));
       const float mxs = mx * sl2;
       float alpha = 1.f;
       if (mxs > m_used + kRescaleLog2) {
@@ -401,9 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
       }
-      // p = 2^(s sigma log2(e) - m): packed fp32x2 FMA, the hardware exp2 for
-      // 11 of 16 pairs and the FMA-pipe cubic for 5; P to TMEM as bf16 pairs
-      // over the first 64 columns of S_x
+      // p = 2^(s sigma log2(e) - m): packed fp32x2 FMA and the hardware exp2
+      // (the FMA-pipe cubic for kPolyPairs of every 16 pairs); P to TMEM as
+      // bf16 pairs over the first 64 columns of S_x, each half signalled as
+      // soon as it is written
       const float2 neg_m2 = make_float2(-mu, -mu);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
@@ -415,18 +439,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 xx = __ffma2_rn(make_float2(__uint_as_float(v[c * 32 + 2 * e]),
                                                    __uint_as_float(v[c * 32 + 2 * e + 1])),
                                        sl2x2, neg_m2);
-          const float2 p = (e % 3 == 2) ? exp2_poly2(xx)
+          const float2 p = poly_pair(e) ? exp2_poly2(xx)
                                         : make_float2(ex2_approx(xx.x), ex2_approx(xx.y));
           acc[e & 3] = __fadd2_rn(acc[e & 3], p);
           pk[e] = pack_bf16(p.x, p.y);
         }
         tmem_st16(tS + c * 16, pk);
+        if (c == 1 || c == 3) {
+          tmem_wait_st();
+          tc_fence_before();
+          warp_arrive(&bar->p_full[x][c >> 1], lane);
+        }
       }
       const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-      tmem_wait_st();
       l = l * alpha + (a.x + a.y);
-      tc_fence_before();
-      warp_arrive(&bar->p_full[x], lane);
     }
     if (ok && !mbar_wait_warp(&bar->o_final[x], 0, s_abort, err, 44)) ok = false;
     bf16 *orow = out + ((size_t)t.bg * dm.n + qrow) * D;

@@ -91,6 +91,13 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // The hardware base-2 exponential (MUFU), flushing subnormals: ex2(-inf) = 0.
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
