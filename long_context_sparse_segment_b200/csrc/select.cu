@@ -15,7 +15,9 @@
 //   then one warp per query block decides, without sorting:
 //   TOPK_FRAC: k = max(1, floor(f * (I + 1))); the t = max(0, k - own)
 //     earlier-segment blocks of largest score (ties: lower J) are found by
-//     bisection over the 64-bit order keys of the scores;
+//     a radix select over the 64-bit order keys of the scores (eight rounds
+//     of 8-bit digit histograms: the t-th largest key and how many of the
+//     keys equal to it are taken);
 //   THRESHOLD: softmax over the admissible blocks; bisection finds the
 //     largest score s such that the own-segment mass plus the mass of the
 //     earlier blocks scoring >= s reaches tau; blocks scoring above s are
@@ -36,8 +38,10 @@ constexpr int kChunk = 64;       // key blocks per staged chunk: 8 warps x 8
 constexpr int kPad = 132;        // doubles per staged row: conflict-free B reads
 constexpr size_t kSmemBudget = 220 * 1024;
 
+constexpr int kWarps = kThreads / 32;
+
 size_t sel_smem(int rows, int nb) {
-  return (size_t)kChunk * kPad * 8 + (size_t)rows * nb * (8 + 8 + 1) + 64;
+  return (size_t)kChunk * kPad * 8 + (size_t)rows * nb * (8 + 8 + 1) + kWarps * 256 * 4 + 64;
 }
 
 int sel_rows(int nb) {
@@ -86,7 +90,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned long long *keys =
       reinterpret_cast<unsigned long long *>(kb + kChunk * kPad);  // [rows][nb]
   double *pis = reinterpret_cast<double *>(keys + (size_t)rows * nb);  // [rows][nb]
-  unsigned char *flags = reinterpret_cast<unsigned char *>(pis + (size_t)rows * nb);
+  unsigned *hists = reinterpret_cast<unsigned *>(pis + (size_t)rows * nb);  // [kWarps][256]
+  unsigned char *flags = reinterpret_cast<unsigned char *>(hists + kWarps * 256);
 
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int bg = blockIdx.y, b = bg / dm.hq, g = bg % dm.hq;
@@ -163,17 +168,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t == f0) {
         all_earlier = true;
       } else if (t > 0) {
-        unsigned long long k = 0;  // largest value with count(key >= value) >= t
-        for (int bit = 63; bit >= 0; --bit) {
-          const unsigned long long cand = k | (1ull << bit);
-          int c = 0;
-          for (int J = lane; J < f0; J += 32) c += key[J] >= cand;
-          if (warp_sum_i(c) >= t) k = cand;
+        // The t-th largest key, one 8-bit digit at a time from the top: among
+        // the keys that share the digits found so far, count each value of
+        // the next digit, and take the digit at which the count from the top
+        // reaches the number still needed.
+        unsigned *hist = hists + w * 256;
+        unsigned long long pre = 0, pmask = 0;
+        int need = t;
+        for (int shift = 56; shift >= 0; shift -= 8) {
+          for (int d = lane; d < 256; d += 32) hist[d] = 0;
+          __syncwarp();
+          for (int J = lane; J < f0; J += 32) {
+            const unsigned long long kj = key[J];
+            if ((kj & pmask) == pre) atomicAdd(&hist[(unsigned)(kj >> shift) & 255u], 1u);
+          }
+          __syncwarp();
+          // lane l holds digits 255 - 8l .. 248 - 8l (descending)
+          unsigned c[8], tot = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) tot += (c[e] = hist[255 - 8 * lane - e]);
+          unsigned incl = tot;  // inclusive prefix over lanes, from digit 255 down
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+          }
+          const unsigned excl = incl - tot;
+          const unsigned hit = __ballot_sync(0xffffffffu, excl < (unsigned)need && incl >= (unsigned)need);
+          const int src = __ffs(hit) - 1;
+          int digit = 0, above = 0;
+          if (lane == src) {
+            unsigned run = excl;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              if (run + c[e] >= (unsigned)need) {
+                digit = 255 - 8 * lane - e;
+                break;
+              }
+              run += c[e];
+            }
+            above = (int)run;
+          }
+          digit = __shfl_sync(0xffffffffu, digit, src);
+          above = __shfl_sync(0xffffffffu, above, src);
+          need -= above;
+          pre |= (unsigned long long)digit << shift;
+          pmask |= 255ull << shift;
+          __syncwarp();
         }
-        int gt = 0;
-        for (int J = lane; J < f0; J += 32) gt += key[J] > k;
-        kcut = k;
-        tie_take = t - warp_sum_i(gt);
+        kcut = pre;
+        tie_take = need;  // keys equal to the cut that are still taken
       }
     } else {
       const double tau = (double)param;
