@@ -40,8 +40,11 @@ constexpr size_t kSmemBudget = 220 * 1024;
 
 constexpr int kWarps = kThreads / 32;
 
+// Score keys are stored with a row stride of nb + 1 words, so that the
+// eight rows of one tensor-core result land in different banks.
 size_t sel_smem(int rows, int nb) {
-  return (size_t)kChunk * kPad * 8 + (size_t)rows * nb * (8 + 8 + 1) + kWarps * 256 * 4 + 64;
+  return (size_t)kChunk * kPad * 8 + (size_t)rows * (nb + 1) * 8 + (size_t)rows * nb * (8 + 1) +
+         kWarps * 256 * 4 + 64;
 }
 
 int sel_rows(int nb) {
@@ -88,8 +91,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nb = dm.nb;
   double *kb = reinterpret_cast<double *>(smem);  // [kChunk][kPad]
   unsigned long long *keys =
-      reinterpret_cast<unsigned long long *>(kb + kChunk * kPad);  // [rows][nb]
-  double *pis = reinterpret_cast<double *>(keys + (size_t)rows * nb);  // [rows][nb]
+      reinterpret_cast<unsigned long long *>(kb + kChunk * kPad);  // [rows][nb + 1]
+  double *pis = reinterpret_cast<double *>(keys + (size_t)rows * (nb + 1));  // [rows][nb]
   unsigned *hists = reinterpret_cast<unsigned *>(pis + (size_t)rows * nb);  // [kWarps][256]
   unsigned char *flags = reinterpret_cast<unsigned char *>(hists + kWarps * 256);
 
@@ -130,17 +133,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncthreads();
       if (c0 + kChunk < max_adm) fetch(c0 + kChunk);
-      double acc[2] = {0.0, 0.0};
+      // four independent accumulation chains over d, added in a fixed order
+      double acc4[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
       const double *brow = kb + (w * 8 + (lane >> 2)) * kPad + (lane & 3);
 #pragma unroll
-      for (int k = 0; k < D / 4; ++k) dmma_8x8x4(acc, a[k], brow[4 * k]);
+      for (int k = 0; k < D / 4; ++k) dmma_8x8x4(acc4[k & 3], a[k], brow[4 * k]);
+      double acc[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) acc[u] = (acc4[0][u] + acc4[1][u]) + (acc4[2][u] + acc4[3][u]);
       if (ar < nrows) {
         const int I = I0 + ar;
         const int adm = min(nb, (I / dm.spb + 1) * dm.spb);
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int J = c0 + w * 8 + 2 * (lane & 3) + u;
-          if (J < adm) keys[(size_t)ar * nb + J] = f64_order_key(sigma * acc[u]);
+          if (J < adm) keys[(size_t)ar * (nb + 1) + J] = f64_order_key(sigma * acc[u]);
         }
       }
     }
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int seg = I / dm.spb;
   const int f0 = seg * dm.spb;  // own segment: [f0, adm); earlier blocks: [0, f0)
   const int adm = min(nb, f0 + dm.spb);
-  const unsigned long long *key = keys + (size_t)w * nb;
+  const unsigned long long *key = keys + (size_t)w * (nb + 1);
   double *pi = pis + (size_t)w * nb;
   unsigned char *flag = flags + (size_t)w * nb;
 
