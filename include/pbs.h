@@ -10,6 +10,7 @@
  *   pbs_select_blocks  key blocks kept per query block, from pooled scores
  *   pbs_attn_fwd       causal block-sparse attention on the permuted keys
  *   pbs_unpermute      inverse permutation of the output rows
+ *   pbs_attn_fwd_unpermute  the last two fused: rows written in place
  *
  * Conventions shared by every call
  * --------------------------------
@@ -213,6 +214,28 @@ pbs_status pbs_attn_fwd(const void *q_or_qperm, const void *k_perm,
                         const int32_t *qpos, const int32_t *blk_idx,
                         const int32_t *blk_cnt, void *out, float *lse,
                         pbs_shape s, float scale, pbs_stream_t st);
+
+/*
+ * pbs_attn_fwd_unpermute - pbs_attn_fwd followed by pbs_unpermute, fused:
+ * each output row is written straight to its query's original position.
+ * Source: skillmd.com "Implementation Steps" (output[argsort(perm)]) and
+ * sciencestack.ai Theorem 3.3, as for the two calls it replaces; the fusion
+ * itself is this library's (the pages run the two steps separately).
+ *
+ * Arguments as for pbs_attn_fwd with the queries in permuted order: row p
+ * of head g (query q_perm[b, g, p], original position qpos[b, g/G, p]) is
+ * written to out[b, g, qpos[b, g/G, p]], and its LSE to lse[b, g, qpos[...]].
+ * With qpos NULL this is pbs_attn_fwd. qpos must hold each segment's
+ * positions once (as written by pbs_permute); a position outside [0, n) is
+ * reported as PBS_ERR_DEVICE_ASSERT and its row is not written. `out` must
+ * not overlap q_perm, k_perm or v_perm (PBS_ERR_INVALID_ARG when it is one
+ * of them).
+ */
+pbs_status pbs_attn_fwd_unpermute(const void *q_perm, const void *k_perm,
+                                  const void *v_perm, const int32_t *kpos,
+                                  const int32_t *qpos, const int32_t *blk_idx,
+                                  const int32_t *blk_cnt, void *out, float *lse,
+                                  pbs_shape s, float scale, pbs_stream_t st);
 
 /*
  * pbs_unpermute - inverse permutation of the output rows.

@@ -161,10 +161,12 @@ pbs_status pbs_select_blocks(const void *q_or_qperm, const void *k_perm, const d
                                    blk_idx, blk_cnt, blk_mask, err, cs));
 }
 
-pbs_status pbs_attn_fwd(const void *q_or_qperm, const void *k_perm, const void *v_perm,
-                        const int32_t *kpos, const int32_t *qpos, const int32_t *blk_idx,
-                        const int32_t *blk_cnt, void *out, float *lse, pbs_shape s, float scale,
-                        pbs_stream_t st) {
+namespace {
+
+pbs_status attn_fwd(const void *q_or_qperm, const void *k_perm, const void *v_perm,
+                    const int32_t *kpos, const int32_t *qpos, const int32_t *blk_idx,
+                    const int32_t *blk_cnt, void *out, float *lse, pbs_shape s, float scale,
+                    bool scatter, pbs_stream_t st) {
   Dims dm;
   pbs_status r = check_shape(s, &dm);
   if (r != PBS_OK) return r;
@@ -175,10 +177,30 @@ pbs_status pbs_attn_fwd(const void *q_or_qperm, const void *k_perm, const void *
       (kpos && !aligned16(kpos)) || (qpos && ((uintptr_t)qpos & 3u)) ||
       ((uintptr_t)blk_idx & 3u) || ((uintptr_t)blk_cnt & 3u) || (lse && ((uintptr_t)lse & 3u)))
     return PBS_ERR_INVALID_ARG;
+  // rows land out of order: the output must not be an input still being read
+  if (scatter && (out == q_or_qperm || out == k_perm || out == v_perm)) return PBS_ERR_INVALID_ARG;
   int *err = error_word();
   const float sigma = (float)resolve_sigma(scale, dm.d);
   return cuda_status(launch_attn(dm, q_or_qperm, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt,
-                                 out, lse, sigma, err, (cudaStream_t)st));
+                                 out, lse, sigma, err, scatter && qpos, (cudaStream_t)st));
+}
+
+}  // namespace
+
+pbs_status pbs_attn_fwd(const void *q_or_qperm, const void *k_perm, const void *v_perm,
+                        const int32_t *kpos, const int32_t *qpos, const int32_t *blk_idx,
+                        const int32_t *blk_cnt, void *out, float *lse, pbs_shape s, float scale,
+                        pbs_stream_t st) {
+  return attn_fwd(q_or_qperm, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt, out, lse, s, scale,
+                  false, st);
+}
+
+pbs_status pbs_attn_fwd_unpermute(const void *q_perm, const void *k_perm, const void *v_perm,
+                                  const int32_t *kpos, const int32_t *qpos,
+                                  const int32_t *blk_idx, const int32_t *blk_cnt, void *out,
+                                  float *lse, pbs_shape s, float scale, pbs_stream_t st) {
+  return attn_fwd(q_perm, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt, out, lse, s, scale, true,
+                  st);
 }
 
 pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out, pbs_shape s,

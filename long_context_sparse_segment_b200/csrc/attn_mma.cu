@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(MmaCfg<D, BB>::kThreads, 1)
                     const bf16 *__restrict__ vp, const int32_t *__restrict__ kpos,
                     const int32_t *__restrict__ qpos, const int32_t *__restrict__ blk_idx,
                     const int32_t *__restrict__ blk_cnt, bf16 *__restrict__ out,
-                    float *__restrict__ lse, Dims dm, float sl2, int *err) {
+                    float *__restrict__ lse, Dims dm, float sl2, int *err, int scatter) {
   using C = MmaCfg<D, BB>;
   extern __shared__ __align__(128) uint8_t smem[];
   bf16 *Qs = reinterpret_cast<bf16 *>(smem);
@@ -211,20 +211,30 @@ __global__ void __launch_bounds__(MmaCfg<D, BB>::kThreads, 1)
   for (int e = 0; e < 2; ++e) {
     const int r = warp * 16 + (lane >> 2) + e * 8;
     const float inv = l[e] > 0.f ? 1.f / l[e] : 0.f;
-    bf16 *orow = out + (qrow0 + r) * D;
+    // the row goes to its place in the given order, or with `scatter` to its
+    // query's original position (the inverse permutation, fused)
+    size_t orow_i = qrow0 + r;
+    if (scatter) {
+      if (qp[e] < 0 || qp[e] >= dm.n) {
+        report(err, PBS_ERR_DEVICE_ASSERT);
+        continue;
+      }
+      orow_i = (size_t)bg * dm.n + qp[e];
+    }
+    bf16 *orow = out + orow_i * D;
 #pragma unroll
     for (int j = 0; j < D / 8; ++j)
       *reinterpret_cast<uint32_t *>(orow + j * 8 + 2 * (lane & 3)) =
           pack_bf16(o[j][e * 2] * inv, o[j][e * 2 + 1] * inv);
     if (lse && (lane & 3) == 0)
-      lse[qrow0 + r] = l[e] > 0.f ? (m[e] + log2f(l[e])) * kLn2 : -INFINITY;
+      lse[orow_i] = l[e] > 0.f ? (m[e] + log2f(l[e])) * kLn2 : -INFINITY;
   }
 }
 
 template <int D, int BB>
 cudaError_t run(const Dims &dm, const void *q, const void *kp, const void *vp,
                 const int32_t *kpos, const int32_t *qpos, const int32_t *idx, const int32_t *cnt,
-                void *out, float *lse, float sigma, int *err, cudaStream_t st) {
+                void *out, float *lse, float sigma, int *err, bool scatter, cudaStream_t st) {
   using C = MmaCfg<D, BB>;
   cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<D, BB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem);
@@ -232,7 +242,7 @@ cudaError_t run(const Dims &dm, const void *q, const void *kp, const void *vp,
   const unsigned grid = (unsigned)dm.b * dm.hq * dm.nb;
   attn_mma_kernel<D, BB><<<grid, C::kThreads, C::smem, st>>>(
       (const bf16 *)q, (const bf16 *)kp, (const bf16 *)vp, kpos, qpos, idx, cnt, (bf16 *)out,
-      lse, dm, sigma * kLog2e, err);
+      lse, dm, sigma * kLog2e, err, scatter ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -241,14 +251,14 @@ cudaError_t run(const Dims &dm, const void *q, const void *kp, const void *vp,
 cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                             const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            cudaStream_t st) {
+                            bool scatter, cudaStream_t st) {
   if (dm.d == 64 && dm.B == 64)
-    return run<64, 64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, st);
+    return run<64, 64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter, st);
   if (dm.d == 64 && dm.B == 128)
-    return run<64, 128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, st);
+    return run<64, 128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter, st);
   if (dm.d == 128 && dm.B == 64)
-    return run<128, 64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, st);
-  return run<128, 128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, st);
+    return run<128, 64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter, st);
+  return run<128, 128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter, st);
 }
 
 }  // namespace pbs
@@ -268,7 +278,7 @@ namespace pbs {
 cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const void *vp,
                         const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                         const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                        cudaStream_t st) {
+                        bool scatter, cudaStream_t st) {
   const char *fwd = getenv("PBS_FORWARD");
   const bool force_mma = fwd && strcmp(fwd, "mma") == 0;
   const bool force_tc1 = fwd && strcmp(fwd, "tc1") == 0;
@@ -277,12 +287,15 @@ cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const voi
     const int fault = (fi && strcmp(fi, "timeout") == 0) ? 1 : 0;
     if (!force_tc1) {
       const cudaError_t e =
-          launch_attn_tc2(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, st);
+          launch_attn_tc2(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+                          scatter, st);
       if (e != cudaErrorInvalidConfiguration) return e;
     }
-    return launch_attn_tc(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, st);
+    return launch_attn_tc(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+                          scatter, st);
   }
-  return launch_attn_mma(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, st);
+  return launch_attn_mma(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter,
+                         st);
 }
 
 }  // namespace pbs

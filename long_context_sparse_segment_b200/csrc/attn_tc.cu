@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ kpos,
                    const int32_t *__restrict__ qpos, const int32_t *__restrict__ blk_idx,
                    const int32_t *__restrict__ blk_cnt, bf16 *__restrict__ out,
-                   float *__restrict__ lse, Dims dm, float sl2, int *err, int fault) {
+                   float *__restrict__ lse, Dims dm, float sl2, int *err, int fault,
+                   int scatter) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>(
@@ -416,7 +417,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       warp_arrive(&bar->lsum, lane);
       if (!mbar_wait_warp(&bar->lsum, 0, s_abort, err, 46)) ok = false;
     }
-    bf16 *orow = out + ((size_t)bg * dm.n + qrow) * D + half * OC;
+    // the row goes to its place in the given order, or with `scatter` to its
+    // query's original position (the inverse permutation, fused)
+    int orow_i = qrow;
+    if (scatter) {
+      orow_i = qp;
+      if (qp < 0 || qp >= dm.n) {
+        report(err, PBS_ERR_DEVICE_ASSERT);
+        ok = false, orow_i = -1;
+      }
+    }
+    bf16 *orow = out + ((size_t)bg * dm.n + (orow_i < 0 ? 0 : orow_i)) * D + half * OC;
     if (ok) {
       const float lt = l + xc->l[half ^ 1][row];
       tc_fence_after();
@@ -436,11 +447,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
       if (lse && half == 0)
-        lse[(size_t)bg * dm.n + qrow] = lt > 0.f ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
-    } else if (count == 0) {
+        lse[(size_t)bg * dm.n + orow_i] = lt > 0.f ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
+    } else if (count == 0 && orow_i >= 0) {
       for (int c = 0; c < OC / 8; ++c)
         reinterpret_cast<uint4 *>(orow)[c] = make_uint4(0, 0, 0, 0);
-      if (lse && half == 0) lse[(size_t)bg * dm.n + qrow] = -INFINITY;
+      if (lse && half == 0) lse[(size_t)bg * dm.n + orow_i] = -INFINITY;
     }
   }
   tc_fence_before();
@@ -455,7 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t run(const Dims &dm, const void *q, const void *kp, const void *vp,
                 const int32_t *kpos, const int32_t *qpos, const int32_t *idx, const int32_t *cnt,
-                void *out, float *lse, float sigma, int *err, int fault, cudaStream_t st) {
+                void *out, float *lse, float sigma, int *err, int fault, bool scatter,
+                cudaStream_t st) {
   CUtensorMap mk, mv;
   if (!make_tile_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D, 128) ||
       !make_tile_map(&mv, vp, (uint64_t)dm.b * dm.hkv * dm.n, D, 128))
@@ -467,7 +479,7 @@ cudaError_t run(const Dims &dm, const void *q, const void *kp, const void *vp,
   const unsigned grid = (unsigned)dm.b * dm.hq * dm.nb;
   attn_tc_kernel<D><<<grid, kThreads, smem, st>>>((const bf16 *)q, mk, mv, kpos, qpos, idx, cnt,
                                                   (bf16 *)out, lse, dm, sigma * kLog2e, err,
-                                                  fault);
+                                                  fault, scatter ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -478,9 +490,10 @@ bool attn_tc_supported(const Dims &dm) { return dm.B == 128 && (dm.d == 128 || d
 cudaError_t launch_attn_tc(const Dims &dm, const void *q, const void *kp, const void *vp,
                            const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                            const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                           int fault, cudaStream_t st) {
-  if (dm.d == 64) return run<64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, st);
-  return run<128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, st);
+                           int fault, bool scatter, cudaStream_t st) {
+  if (dm.d == 64)
+    return run<64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, scatter, st);
+  return run<128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, scatter, st);
 }
 
 }  // namespace pbs

@@ -142,7 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ kpos,
                     const int32_t *__restrict__ qpos, const int32_t *__restrict__ blk_idx,
                     const int32_t *__restrict__ blk_cnt, bf16 *__restrict__ out,
-                    float *__restrict__ lse, Dims dm, float sl2, int *err, int fault) {
+                    float *__restrict__ lse, Dims dm, float sl2, int *err, int fault,
+                    int scatter) {
   using C = Cfg2<D>;
   constexpr int KS = C::KS, VS = C::VS;
   extern __shared__ uint8_t smem_raw[];
@@ -455,7 +456,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       l = l * alpha + (a.x + a.y);
     }
     if (ok && !mbar_wait_warp(&bar->o_final[x], 0, s_abort, err, 44)) ok = false;
-    bf16 *orow = out + ((size_t)t.bg * dm.n + qrow) * D;
+    // the row goes to its place in the given order, or with `scatter` to its
+    // query's original position (the inverse permutation, fused)
+    int orow_i = qrow;
+    if (scatter) {
+      orow_i = qp;
+      if (qp < 0 || qp >= dm.n) {
+        report(err, PBS_ERR_DEVICE_ASSERT);
+        ok = false, orow_i = -1;
+      }
+    }
+    bf16 *orow = out + ((size_t)t.bg * dm.n + (orow_i < 0 ? 0 : orow_i)) * D;
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -474,10 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
       }
       if (lse)
-        lse[(size_t)t.bg * dm.n + qrow] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
-    } else if (valid && t.count == 0) {
+        lse[(size_t)t.bg * dm.n + orow_i] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+    } else if (valid && t.count == 0 && orow_i >= 0) {
       for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(orow)[c] = make_uint4(0, 0, 0, 0);
-      if (lse) lse[(size_t)t.bg * dm.n + qrow] = -INFINITY;
+      if (lse) lse[(size_t)t.bg * dm.n + orow_i] = -INFINITY;
     }
     tc_fence_before();
     __syncthreads();
@@ -487,7 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t run2(const Dims &dm, const void *q, const void *kp, const void *vp,
                  const int32_t *kpos, const int32_t *qpos, const int32_t *idx, const int32_t *cnt,
-                 void *out, float *lse, float sigma, int *err, int fault, cudaStream_t st) {
+                 void *out, float *lse, float sigma, int *err, int fault, bool scatter,
+                 cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_tile_map(&mq, q, (uint64_t)dm.b * dm.hq * dm.n, D, kBM) ||
       !make_tile_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D, kBN) ||
@@ -506,7 +518,8 @@ cudaError_t run2(const Dims &dm, const void *q, const void *kp, const void *vp,
   const long long total = (long long)dm.b * dm.hq * dm.nb;
   const unsigned grid = (unsigned)((total + 1) / 2);
   attn_tc2_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, kpos, qpos, idx, cnt, (bf16 *)out,
-                                                   lse, dm, sigma * kLog2e, err, fault);
+                                                   lse, dm, sigma * kLog2e, err, fault,
+                                                   scatter ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -515,9 +528,10 @@ cudaError_t run2(const Dims &dm, const void *q, const void *kp, const void *vp,
 cudaError_t launch_attn_tc2(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                             const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            int fault, cudaStream_t st) {
-  if (dm.d == 64) return run2<64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, st);
-  return run2<128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, st);
+                            int fault, bool scatter, cudaStream_t st) {
+  if (dm.d == 64)
+    return run2<64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, scatter, st);
+  return run2<128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, scatter, st);
 }
 
 }  // namespace pbs

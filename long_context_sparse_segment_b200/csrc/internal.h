@@ -44,30 +44,31 @@ cudaError_t launch_select(const Dims &dm, const double *qsum, const double *ksum
                           float param, double sigma, int32_t *idx, int32_t *cnt,
                           uint8_t *mask, int *err, cudaStream_t st);
 
-// block-sparse forward
+// block-sparse forward; with `scatter` each output row is written at its
+// query's original position (qpos) instead of its place in the given order
 cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const void *vp,
                         const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                         const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                        cudaStream_t st);
+                        bool scatter, cudaStream_t st);
 
 // the forward on the tcgen05 tensor cores (B = 128, d in {64, 128})
 bool attn_tc_supported(const Dims &dm);
 cudaError_t launch_attn_tc(const Dims &dm, const void *q, const void *kp, const void *vp,
                            const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                            const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                           int fault, cudaStream_t st);
+                           int fault, bool scatter, cudaStream_t st);
 
 // the same forward with two query tiles per CTA (tcgen05; B = 128, d in {64, 128})
 cudaError_t launch_attn_tc2(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                             const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            int fault, cudaStream_t st);
+                            int fault, bool scatter, cudaStream_t st);
 
 // the same forward on the legacy warp-MMA path
 cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                             const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            cudaStream_t st);
+                            bool scatter, cudaStream_t st);
 
 // out[qpos[p]] = out_perm[p]
 cudaError_t launch_unpermute(const Dims &dm, const void *op, const int32_t *qpos, void *out,

@@ -68,11 +68,6 @@ __device__ __forceinline__ double warp_max_d(double v) {
   for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
-__device__ __forceinline__ int warp_sum_i(int v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 // D[8x8] += A[8x4] * B[4x8] in fp64: lane t holds A[t/4][t%4], B[t%4][t/4],
 // D[t/4][2(t%4)] and D[t/4][2(t%4)+1].

@@ -114,9 +114,11 @@ def select_blocks(q, k_perm, kbar_sum, block, segment, mode, param=0.0, scale=0.
 
 
 def attn_fwd(q, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt, block, segment, scale=0.0,
-             lse=False, out=None):
+             lse=False, out=None, unpermute=False):
     """Block-sparse causal attention over the permuted keys: o [b,hq,n,d] bf16
-    (and lse [b,hq,n] fp32 when asked)."""
+    (and lse [b,hq,n] fp32 when asked). With ``unpermute`` (permuted queries)
+    each row is written at its query's original position in the same call
+    (pbs_attn_fwd_unpermute) instead of in the order of ``q``."""
     _need(q, "q", torch.bfloat16)
     _need(k_perm, "k_perm", torch.bfloat16, q.device)
     _need(v_perm, "v_perm", torch.bfloat16, q.device)
@@ -128,9 +130,10 @@ def attn_fwd(q, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt, block, segment, sc
     shp = shape_of(q, k_perm, block, segment)
     o = out if out is not None else torch.empty_like(q)
     l = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if lse else None
-    check(lib().pbs_attn_fwd(_ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(kpos), _ptr(qpos),
-                             _ptr(blk_idx), _ptr(blk_cnt), _ptr(o), _ptr(l), shp, scale,
-                             _stream(q.device)), "pbs_attn_fwd")
+    fn = lib().pbs_attn_fwd_unpermute if unpermute else lib().pbs_attn_fwd
+    check(fn(_ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(kpos), _ptr(qpos), _ptr(blk_idx),
+             _ptr(blk_cnt), _ptr(o), _ptr(l), shp, scale, _stream(q.device)),
+          "pbs_attn_fwd_unpermute" if unpermute else "pbs_attn_fwd")
     return (o, l) if lse else o
 
 
@@ -157,19 +160,26 @@ def device_status(device=None, detail=False):
 
 
 def pbs_attention(q, k, v, block, segment, mode="threshold", param=0.9, scale=0.0,
-                  permute_q=False, keep=False):
+                  permute_q=False, keep=False, fused_unpermute=True):
     """The whole prefill path: score -> permute -> select -> attend ->
     unpermute. Returns o [b, hq, n, d] bf16 in the natural query order, or a
-    dict with every intermediate when ``keep`` is true."""
+    dict with every intermediate when ``keep`` is true. In permuted-query
+    mode the last two steps are one call unless ``fused_unpermute`` is
+    false (then ``o_perm`` holds the rows in permuted order)."""
     imp = score(q, k, block, segment, scale)
     perm = permute(imp, k, v, block, segment, q=q if permute_q else None, hq=q.shape[1])
     q_used = perm["q_perm"] if permute_q else q
     qpos = perm["kpos"] if permute_q else None
     idx, cnt, _ = select_blocks(q_used, perm["k_perm"], perm["kbar_sum"], block, segment, mode,
                                 param, scale)
-    o_perm = attn_fwd(q_used, perm["k_perm"], perm["v_perm"], perm["kpos"], qpos, idx, cnt,
-                      block, segment, scale)
-    o = unpermute(o_perm, qpos, k.shape[1], block, segment) if permute_q else o_perm
+    if permute_q and fused_unpermute:
+        o = attn_fwd(q_used, perm["k_perm"], perm["v_perm"], perm["kpos"], qpos, idx, cnt,
+                     block, segment, scale, unpermute=True)
+        o_perm = None
+    else:
+        o_perm = attn_fwd(q_used, perm["k_perm"], perm["v_perm"], perm["kpos"], qpos, idx, cnt,
+                          block, segment, scale)
+        o = unpermute(o_perm, qpos, k.shape[1], block, segment) if permute_q else o_perm
     if keep:
         return dict(perm, imp=imp, idx=idx, cnt=cnt, o_perm=o_perm, o=o, qpos=qpos)
     return o

@@ -285,3 +285,48 @@ def test_two_tile_and_one_tile_forwards_agree(name, permute_q, dev, monkeypatch)
     assert_outputs_close(f64(o1), ref, "one-tile")
     assert_outputs_close(f64(o2), f64(o1), "two-tile vs one-tile")
     np.testing.assert_allclose(f64(lse2), f64(lse1), atol=1e-4)
+
+
+@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128", "odd_items", "d128_b64", "s_eq_n"])
+@pytest.mark.parametrize("forward", ["default", "tc1", "mma"])
+def test_fused_unpermute_equals_two_calls(name, forward, dev, monkeypatch):
+    """pbs_attn_fwd_unpermute writes each row at its query's original
+    position: bit for bit the output of pbs_attn_fwd followed by
+    pbs_unpermute, with the LSE moved the same way."""
+    w = CASES[name]
+    if forward != "default":
+        monkeypatch.setenv("PBS_FORWARD", forward)
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    imp = pbs.score(qd, kd, B)
+    perm = pbs.permute(imp, kd, vd, B, S, q=qd, hq=w.hq)
+    idx, cnt, _ = pbs.select_blocks(perm["q_perm"], perm["k_perm"], perm["kbar_sum"], B, S,
+                                    w.mode, w.param)
+    args = (perm["q_perm"], perm["k_perm"], perm["v_perm"], perm["kpos"], perm["kpos"], idx, cnt,
+            B, S)
+    o_perm, lse_perm = pbs.attn_fwd(*args, lse=True)
+    o_two = pbs.unpermute(o_perm, perm["kpos"], w.hkv, B, S)
+    o_one, lse_one = pbs.attn_fwd(*args, lse=True, unpermute=True)
+    torch.cuda.synchronize()
+    assert pbs.device_status() == 0
+    assert torch.equal(o_one, o_two)
+    qpos = np.repeat(i64(perm["kpos"]), w.group, axis=1)
+    lse_two = np.empty_like(f64(lse_perm))
+    np.put_along_axis(lse_two, qpos, f64(lse_perm), axis=2)
+    np.testing.assert_array_equal(f64(lse_one), lse_two)
+    # and the path entry point uses it
+    o_path = pbs.pbs_attention(qd, kd, vd, B, S, w.mode, w.param, permute_q=True)
+    assert torch.equal(o_path, o_one)
+
+
+def test_fused_unpermute_rejects_output_aliasing_an_input(dev):
+    w = CASES["gqa2k"]
+    _, (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    imp = pbs.score(qd, kd, B)
+    perm = pbs.permute(imp, kd, vd, B, S, q=qd, hq=w.hq)
+    idx, cnt, _ = pbs.select_blocks(perm["q_perm"], perm["k_perm"], perm["kbar_sum"], B, S,
+                                    w.mode, w.param)
+    with pytest.raises(pbs.PbsError):
+        pbs.attn_fwd(perm["q_perm"], perm["k_perm"], perm["v_perm"], perm["kpos"], perm["kpos"],
+                     idx, cnt, B, S, out=perm["q_perm"], unpermute=True)
