@@ -260,8 +260,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(fault == 1 && t == 0)) mbar_wait(&bar->k_full[t % KS], (t / KS) & 1, &never, nullptr);
     for (int t = vseq > VS ? vseq - VS : 0; t < vseq; ++t)
       mbar_wait(&bar->v_full[t % VS], (t / VS) & 1, &never, nullptr);
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // -------------------------------------------------------- MMA issue
+    // The whole warp runs the loop (waits and descriptor arithmetic stay
+    // warp-uniform); one elected lane issues every MMA and every commit.
+    const bool leader = elect_one();
     constexpr uint32_t kIdQK = idesc_bf16(kBM, kBN, false);
     constexpr uint32_t kIdPV = idesc_bf16(kBM, D, true);
     const uint32_t hi = sw128_desc_hi(1024);
@@ -269,21 +272,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lo_k = sw128_desc_lo(smem_u32(sK), 16);
     const uint32_t lo_v = sw128_desc_lo(smem_u32(sV), C::HALF);
     int ks = 0, kph = 0, vs = 0, vph = 0;
-    bool ok = cmax > 0 && mbar_wait(&bar->q_full, 0, s_abort, err, 31);
+    bool ok = cmax > 0 && mbar_wait_warp(&bar->q_full, 0, s_abort, err, 31);
     if (ok) tc_fence_after();
     // S_x = Q_x K'^T: A = Q_x, B = the K' tile, both K-major in shared memory
     auto qk = [&](int x) -> bool {
-      if (!mbar_wait(&bar->k_full[ks], kph, s_abort, err, 32)) return false;
+      if (!mbar_wait_warp(&bar->k_full[ks], kph, s_abort, err, 32)) return false;
       tc_fence_after();
       const uint32_t lq = lo_q + x * (C::TILE >> 4), lk = lo_k + ks * (C::TILE >> 4);
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t step = ((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4;
-        mma_ss(tbase + x * 128, desc_words(lq + step, hi), desc_words(lk + step, hi), kIdQK,
-               kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t step = ((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4;
+          mma_ss(tbase + x * 128, desc_words(lq + step, hi), desc_words(lk + step, hi), kIdQK,
+                 kk > 0);
+        }
+        mma_commit(&bar->k_empty[ks]);
+        mma_commit(&bar->s_full[x]);
       }
-      mma_commit(&bar->k_empty[ks]);
-      mma_commit(&bar->s_full[x]);
+      __syncwarp();
       if (++ks == KS) ks = 0, kph ^= 1;
       return true;
     };
@@ -292,20 +298,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // The first half of P (keys 0-63) is consumed while the softmax still
     // writes the second.
     auto pv = [&](int x, int j) -> bool {
-      if (!mbar_wait(&bar->p_full[x][0], j & 1, s_abort, err, 33)) return false;
-      if (!mbar_wait(&bar->v_full[vs], vph, s_abort, err, 34)) return false;
+      if (!mbar_wait_warp(&bar->p_full[x][0], j & 1, s_abort, err, 33)) return false;
+      if (!mbar_wait_warp(&bar->v_full[vs], vph, s_abort, err, 34)) return false;
       tc_fence_after();
       const uint32_t lv = lo_v + vs * (C::TILE >> 4);
-#pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk) {
-        if (kk == kBN / 32) {
-          if (!mbar_wait(&bar->p_full[x][1], j & 1, s_abort, err, 35)) return false;
+      for (int h = 0; h < 2; ++h) {
+        if (h == 1) {
+          if (!mbar_wait_warp(&bar->p_full[x][1], j & 1, s_abort, err, 35)) return false;
           tc_fence_after();
         }
-        mma_ts(tbase + 256 + x * 128, tbase + x * 128 + kk * 8,
-               desc_words(lv + kk * (2048 >> 4), hi), kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+        if (leader) {
+#pragma unroll
+          for (int k2 = 0; k2 < kBN / 32; ++k2) {
+            const int kk = h * (kBN / 32) + k2;
+            mma_ts(tbase + 256 + x * 128, tbase + x * 128 + kk * 8,
+                   desc_words(lv + kk * (2048 >> 4), hi), kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        __syncwarp();
       }
-      mma_commit(&bar->v_empty[vs]);
+      if (leader) mma_commit(&bar->v_empty[vs]);
+      __syncwarp();
       if (++vs == VS) vs = 0, vph ^= 1;
       return true;
     };
@@ -317,13 +330,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= c) continue;
         ok = pv(x, j);
         if (!ok) break;
-        if (j + 1 < c)
+        if (j + 1 < c) {
           ok = qk(x);
-        else
-          mma_commit(&bar->o_final[x]);  // O_x is complete once this lands
+        } else {
+          if (leader) mma_commit(&bar->o_final[x]);  // O_x is complete once this lands
+          __syncwarp();
+        }
       }
     // drain: every MMA issued here completes before TMEM is released
-    mma_commit(&bar->mma_done);
+    if (leader) mma_commit(&bar->mma_done);
+    __syncwarp();
     int never = 0;
     mbar_wait(&bar->mma_done, 0, &never, nullptr);
   }

@@ -91,6 +91,16 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// True in exactly one lane of the (converged, full) warp: the issuing lane
+// of a warp that runs a single-thread role with warp-uniform control flow.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // max(a, b, c) in one instruction (three-input max.f32, sm_100).
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
