@@ -195,50 +195,63 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
   // =============================================== warpgroup 0: TMA and MMA
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------- TMA loads
     // Order: K'_A(0), K'_B(0), then per block j and tile x: V'_x(j),
     // K'_x(j+1) -- the tensor core's order, so that a load only ever waits
-    // for a slot that an earlier product frees.
+    // for a slot that an earlier product frees. The whole warp runs the loop;
+    // one elected lane issues the copies.
+    const bool leader = elect_one();
     bool q_issued = false;
     int kseq = 0, vseq = 0;
     if (cmax > 0) {
       prefetch_map(&tmQ);
       prefetch_map(&tmK);
       prefetch_map(&tmV);
-      mbar_expect_tx(&bar->q_full, ((cA > 0) + (cB > 0)) * C::TILE);
-      for (int x = 0; x < 2; ++x) {
-        const Tile &t = x ? tB : tA;
-        if (t.count == 0) continue;
-        for (int h = 0; h < C::H; ++h)
-          tma_load_2d(sQ + x * C::TILE + h * C::HALF, &tmQ, &bar->q_full, h * 64,
-                      t.bg * dm.n + t.I * kBM);
+      if (leader) {
+        mbar_expect_tx(&bar->q_full, ((cA > 0) + (cB > 0)) * C::TILE);
+        for (int x = 0; x < 2; ++x) {
+          const Tile &t = x ? tB : tA;
+          if (t.count == 0) continue;
+          for (int h = 0; h < C::H; ++h)
+            tma_load_2d(sQ + x * C::TILE + h * C::HALF, &tmQ, &bar->q_full, h * 64,
+                        t.bg * dm.n + t.I * kBM);
+        }
       }
+      __syncwarp();
       q_issued = true;
       auto load_k = [&](const Tile &t, int j) -> bool {
         const int s = kseq % KS, u = kseq / KS;
-        if (u > 0 && !mbar_wait(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 11)) return false;
-        const int J = checked_block(t, j, dm, err);
-        mbar_expect_tx(&bar->k_full[s], C::TILE);
-        if (!(fault == 1 && kseq == 0))
-          for (int h = 0; h < C::H; ++h)
-            tma_load_2d(sK + s * C::TILE + h * C::HALF, &tmK, &bar->k_full[s], h * 64,
-                        t.bh * dm.n + J * kBN);
+        if (u > 0 && !mbar_wait_warp(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 11))
+          return false;
+        const int J = checked_block(t, j, dm, leader ? err : nullptr);
+        if (leader) {
+          mbar_expect_tx(&bar->k_full[s], C::TILE);
+          if (!(fault == 1 && kseq == 0))
+            for (int h = 0; h < C::H; ++h)
+              tma_load_2d(sK + s * C::TILE + h * C::HALF, &tmK, &bar->k_full[s], h * 64,
+                          t.bh * dm.n + J * kBN);
+        }
+        __syncwarp();
         ++kseq;
         return true;
       };
       auto load_v = [&](const Tile &t, int j) -> bool {
         const int s = vseq % VS, u = vseq / VS;
-        if (u > 0 && !mbar_wait(&bar->v_empty[s], (u - 1) & 1, s_abort, err, 21)) return false;
-        const int J = checked_block(t, j, dm, err);
+        if (u > 0 && !mbar_wait_warp(&bar->v_empty[s], (u - 1) & 1, s_abort, err, 21))
+          return false;
+        const int J = checked_block(t, j, dm, leader ? err : nullptr);
         const bool with_pos = kpos && J / dm.spb == t.segI;
-        mbar_expect_tx(&bar->v_full[s], C::TILE + (with_pos ? kBN * 4 : 0));
-        for (int h = 0; h < C::H; ++h)
-          tma_load_2d(sV + s * C::TILE + h * C::HALF, &tmV, &bar->v_full[s], h * 64,
-                      t.bh * dm.n + J * kBN);
-        if (with_pos)
-          bulk_load(sKP + s * kBN, kpos + (size_t)t.bh * dm.n + (size_t)J * kBN, kBN * 4,
-                    &bar->v_full[s]);
+        if (leader) {
+          mbar_expect_tx(&bar->v_full[s], C::TILE + (with_pos ? kBN * 4 : 0));
+          for (int h = 0; h < C::H; ++h)
+            tma_load_2d(sV + s * C::TILE + h * C::HALF, &tmV, &bar->v_full[s], h * 64,
+                        t.bh * dm.n + J * kBN);
+          if (with_pos)
+            bulk_load(sKP + s * kBN, kpos + (size_t)t.bh * dm.n + (size_t)J * kBN, kBN * 4,
+                      &bar->v_full[s]);
+        }
+        __syncwarp();
         ++vseq;
         return true;
       };
