@@ -101,13 +101,6 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-// max(a, b, c) in one instruction (three-input max.f32, sm_100).
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // The hardware base-2 exponential (MUFU), flushing subnormals: ex2(-inf) = 0.
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
