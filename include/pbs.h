@@ -11,6 +11,7 @@
  *   pbs_attn_fwd       causal block-sparse attention on the permuted keys
  *   pbs_unpermute      inverse permutation of the output rows
  *   pbs_attn_fwd_unpermute  the last two fused: rows written in place
+ *   pbs_attention_host the whole path on host buffers, copies overlapped
  *
  * Conventions shared by every call
  * --------------------------------
@@ -76,7 +77,8 @@ typedef enum {
   PBS_OP_PERMUTE = 1,
   PBS_OP_SELECT = 2,
   PBS_OP_ATTN = 3,
-  PBS_OP_UNPERMUTE = 4
+  PBS_OP_UNPERMUTE = 4,
+  PBS_OP_HOST_PATH = 5 /* pbs_attention_host */
 } pbs_op;
 
 /* Bytes of device workspace the call `op` needs for shape `s` (0 if none). */
@@ -251,6 +253,39 @@ pbs_status pbs_attn_fwd_unpermute(const void *q_perm, const void *k_perm,
  */
 pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out,
                          pbs_shape s, pbs_stream_t st);
+
+/*
+ * pbs_attention_host - the whole path (score, permute, select, forward; the
+ * queries in natural order) on HOST buffers, with the host-device copies
+ * overlapped with the compute.
+ * Source: the five steps as documented above; the pipelining is this
+ * library's (the pages do not treat host buffers).
+ *
+ * The work is split by KV group (batch b, KV head h: query heads
+ * h*G .. h*G+G-1): the copy of group i+1 into the device (on `h2d`) and of
+ * group i-1 back to the host (on `d2h`) run while group i is computed (on
+ * `compute`), in two device slots of the workspace used in turn. Work
+ * issued later on `compute` is ordered after the last copy to the host, so
+ * synchronising `compute` makes `out` valid. `h2d` and `d2h` may be the same
+ * stream (the copies then run one after the other) but must differ from
+ * `compute` for any overlap. Results equal those of the per-step calls on
+ * the same data up to the order of fp32 sums in the importance (the scoring
+ * passes split the keys differently for one group than for all).
+ *
+ *   q, out       host [batch, hq, n, d] bf16 (page-locked memory for
+ *                asynchronous copies; pageable memory works, slower)
+ *   k, v         host [batch, hkv, n, d] bf16
+ *   mode, param  as for pbs_select_blocks
+ *   ws           device workspace of pbs_workspace_bytes(s, PBS_OP_HOST_PATH)
+ *                bytes (two slots of one KV group's buffers)
+ * Returns PBS_ERR_UNSUPPORTED when the scoring step does not support the
+ * group shape (see pbs_score).
+ */
+pbs_status pbs_attention_host(const void *q, const void *k, const void *v,
+                              void *out, pbs_shape s, int mode, float param,
+                              float scale, void *ws, size_t ws_bytes,
+                              pbs_stream_t compute, pbs_stream_t h2d,
+                              pbs_stream_t d2h);
 
 /*
  * Synchronises `st`, returns in *code the current device's error word

@@ -13,11 +13,11 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_ASSERT, 
 # pbs_sel_mode
 SEL = {"threshold": 0, "topk_frac": 1, "all": 2, "dense_causal": 3}
 # pbs_op
-OP_SCORE, OP_PERMUTE, OP_SELECT, OP_ATTN, OP_UNPERMUTE = range(5)
+OP_SCORE, OP_PERMUTE, OP_SELECT, OP_ATTN, OP_UNPERMUTE, OP_HOST_PATH = range(6)
 
 # every entry point declared in include/pbs.h
 EXPORTS = ("pbs_workspace_bytes", "pbs_score", "pbs_score_static", "pbs_permute", "pbs_select_blocks",
-           "pbs_attn_fwd", "pbs_unpermute", "pbs_attn_fwd_unpermute", "pbs_get_device_status", "pbs_status_string",
+           "pbs_attn_fwd", "pbs_unpermute", "pbs_attn_fwd_unpermute", "pbs_attention_host", "pbs_get_device_status", "pbs_status_string",
            "pbs_version")
 
 
@@ -43,6 +43,8 @@ _SIGS = {
     "pbs_attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, Shape, _f, _vp]),
     "pbs_unpermute": (_i, [_vp, _vp, _vp, Shape, _vp]),
     "pbs_attn_fwd_unpermute": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, Shape, _f, _vp]),
+    "pbs_attention_host": (_i, [_vp, _vp, _vp, _vp, Shape, _i, _f, _f, _vp, _sz,
+                                _vp, _vp, _vp]),
     "pbs_get_device_status": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "pbs_status_string": (ctypes.c_char_p, [_i]),
     "pbs_version": (ctypes.c_char_p, []),

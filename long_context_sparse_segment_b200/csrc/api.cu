@@ -64,6 +64,58 @@ double resolve_sigma(float scale, int d) {
   return scale > 0.f ? (double)scale : 1.0 / sqrt((double)d);
 }
 
+// ------------------------------------------- the host-buffer path's slots
+// pbs_attention_host works one KV group (batch b, KV head h: its G query
+// heads) at a time, in two device slots used in turn.
+constexpr size_t kSlotAlign = 256;
+size_t aup(size_t x) { return (x + kSlotAlign - 1) & ~(kSlotAlign - 1); }
+
+Dims group_dims(const Dims &dm) {
+  Dims g = dm;
+  g.b = 1;
+  g.hq = dm.G;
+  g.hkv = 1;
+  return g;
+}
+
+struct Slot {
+  void *q, *k, *v, *kp, *vp, *o, *score_ws;
+  float *imp;
+  int32_t *kpos, *idx, *cnt;
+  double *kbar, *qsum;
+};
+
+// Lays a slot out from `base` (256-byte aligned); returns its size.
+size_t carve_slot(uint8_t *base, const Dims &g, Slot *sl) {
+  const size_t qb = (size_t)g.hq * g.n * g.d * 2, kb = (size_t)g.n * g.d * 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t *p = base ? base + off : nullptr;
+    off += aup(bytes);
+    return p;
+  };
+  Slot t;
+  t.q = take(qb);
+  t.o = take(qb);
+  t.k = take(kb);
+  t.v = take(kb);
+  t.kp = take(kb);
+  t.vp = take(kb);
+  t.imp = (float *)take((size_t)g.n * 4);
+  t.kpos = (int32_t *)take((size_t)g.n * 4);
+  t.kbar = (double *)take((size_t)g.nb * g.d * 8);
+  t.idx = (int32_t *)take((size_t)g.hq * g.nb * g.nb * 4);
+  t.cnt = (int32_t *)take((size_t)g.hq * g.nb * 4);
+  t.score_ws = take(score_ws_bytes(g));
+  t.qsum = (double *)take(select_ws_bytes(g, false));
+  if (sl) *sl = t;
+  return off;
+}
+
+size_t host_path_ws_bytes(const Dims &dm) {
+  return 2 * carve_slot(nullptr, group_dims(dm), nullptr) + kSlotAlign;
+}
+
 }  // namespace
 }  // namespace pbs
 
@@ -79,6 +131,8 @@ size_t pbs_workspace_bytes(pbs_shape s, int op) {
       return score_ws_bytes(dm);
     case PBS_OP_SELECT:
       return select_ws_bytes(dm, true);
+    case PBS_OP_HOST_PATH:
+      return host_path_ws_bytes(dm);
     default:
       return 0;
   }
@@ -220,6 +274,79 @@ pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out, p
   }
   if (out == out_perm) return PBS_ERR_INVALID_ARG;
   return cuda_status(launch_unpermute(dm, out_perm, qpos, out, error_word(), cs));
+}
+
+pbs_status pbs_attention_host(const void *q, const void *k, const void *v, void *out,
+                              pbs_shape s, int mode, float param, float scale, void *ws,
+                              size_t ws_bytes, pbs_stream_t compute, pbs_stream_t h2d,
+                              pbs_stream_t d2h) {
+  Dims dm;
+  pbs_status r = check_shape(s, &dm);
+  if (r != PBS_OK) return r;
+  if (mode < PBS_SEL_THRESHOLD || mode > PBS_SEL_DENSE_CAUSAL) return PBS_ERR_INVALID_ARG;
+  const bool scored = mode == PBS_SEL_THRESHOLD || mode == PBS_SEL_TOPK_FRAC;
+  if (scored && !(param > 0.f && param <= 1.f)) return PBS_ERR_INVALID_ARG;
+  if (empty(dm)) return PBS_OK;
+  if (!q || !k || !v || !out || !ws) return PBS_ERR_INVALID_ARG;
+  const Dims g = group_dims(dm);
+  if (!score_supported(g)) return PBS_ERR_UNSUPPORTED;
+  if (ws_bytes < host_path_ws_bytes(dm)) return PBS_ERR_WORKSPACE;
+  uint8_t *base = (uint8_t *)(((uintptr_t)ws + kSlotAlign - 1) & ~(uintptr_t)(kSlotAlign - 1));
+  Slot slot[2];
+  const size_t slot_bytes = carve_slot(base, g, &slot[0]);
+  carve_slot(base + slot_bytes, g, &slot[1]);
+
+  cudaStream_t cs = (cudaStream_t)compute, hs = (cudaStream_t)h2d, ds = (cudaStream_t)d2h;
+  cudaEvent_t ev[3][2] = {};  // [copied in, computed, copied out][slot]
+  for (auto &row : ev)
+    for (auto &e : row)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+        for (auto &r2 : ev)
+          for (auto &e2 : r2)
+            if (e2) cudaEventDestroy(e2);
+        return PBS_ERR_CUDA;
+      }
+  int *err = error_word();
+  const float sigma_f = (float)resolve_sigma(scale, dm.d);
+  const double sigma_d = resolve_sigma(scale, dm.d);
+  const size_t qb = (size_t)g.hq * g.n * g.d * 2, kb = (size_t)g.n * g.d * 2;
+  const int groups = dm.b * dm.hkv;
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < groups && e == cudaSuccess; ++i) {
+    const int sid = i & 1, bi = i / dm.hkv, h = i % dm.hkv;
+    const Slot &sl = slot[sid];
+    const size_t qoff = ((size_t)bi * dm.hq + (size_t)h * dm.G) * qb / g.hq;
+    const size_t koff = ((size_t)bi * dm.hkv + h) * kb;
+    // in: the slot is free once group i - 2 has been copied out
+    if (i >= 2) e = cudaStreamWaitEvent(hs, ev[2][sid], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sl.q, (const uint8_t *)q + qoff, qb, cudaMemcpyHostToDevice, hs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sl.k, (const uint8_t *)k + koff, kb, cudaMemcpyHostToDevice, hs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sl.v, (const uint8_t *)v + koff, kb, cudaMemcpyHostToDevice, hs);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[0][sid], hs);
+    // the five steps on the group
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev[0][sid], 0);
+    if (e == cudaSuccess) e = launch_score(g, sl.q, sl.k, sl.imp, sigma_f, sl.score_ws, err, cs);
+    if (e == cudaSuccess) e = launch_segsort(g, sl.imp, sl.kpos, err, cs);
+    if (e == cudaSuccess)
+      e = launch_gather(g, sl.kpos, sl.k, sl.v, nullptr, sl.kp, sl.vp, nullptr, sl.kbar, err, cs);
+    if (e == cudaSuccess && scored) e = launch_blocksum(g, g.hq, sl.q, sl.qsum, cs);
+    if (e == cudaSuccess)
+      e = launch_select(g, sl.qsum, sl.kbar, mode, param, sigma_d, sl.idx, sl.cnt, nullptr, err, cs);
+    if (e == cudaSuccess)
+      e = launch_attn(g, sl.q, sl.kp, sl.vp, sl.kpos, nullptr, sl.idx, sl.cnt, sl.o, nullptr,
+                      sigma_f, err, false, cs);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[1][sid], cs);
+    // out
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ds, ev[1][sid], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync((uint8_t *)out + qoff, sl.o, qb, cudaMemcpyDeviceToHost, ds);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[2][sid], ds);
+  }
+  // work queued on the copy streams is ordered before later work on `compute`
+  for (int sid = 0; sid < 2 && sid < groups && e == cudaSuccess; ++sid)
+    e = cudaStreamWaitEvent(cs, ev[2][sid], 0);
+  for (auto &row : ev)
+    for (auto &ee : row) cudaEventDestroy(ee);  // released once their work completes
+  return cuda_status(e);
 }
 
 pbs_status pbs_get_device_status(pbs_stream_t st, int *code, int *detail) {

@@ -183,3 +183,41 @@ def pbs_attention(q, k, v, block, segment, mode="threshold", param=0.9, scale=0.
     if keep:
         return dict(perm, imp=imp, idx=idx, cnt=cnt, o_perm=o_perm, o=o, qpos=qpos)
     return o
+
+
+_COPY_STREAMS = {}
+
+
+def _copy_streams(device):
+    """Two copy streams per device (host to device, device to host), kept
+    for the life of the process."""
+    key = device.index
+    if key not in _COPY_STREAMS:
+        _COPY_STREAMS[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device))
+    return _COPY_STREAMS[key]
+
+
+def attention_host(q, k, v, block, segment, mode="threshold", param=0.9, scale=0.0, out=None,
+                   device=None, ws=None):
+    """The whole path on host tensors (pbs_attention_host): q [b, hq, n, d],
+    k, v [b, hkv, n, d] bf16 on the CPU (page-locked for overlapped copies);
+    returns o [b, hq, n, d] bf16 on the CPU, valid once the device's current
+    stream is synchronised. The copies run on two library-owned streams and
+    overlap the compute, one KV group at a time."""
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        if t.device.type != "cpu" or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{nm}: contiguous bf16 CPU tensor expected")
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    b, hq, n, d = q.shape
+    shp = Shape(b, hq, k.shape[1], n, d, block, segment)
+    o = out if out is not None else torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    need = workspace_bytes(shp, _lib.OP_HOST_PATH)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    h2d, d2h = _copy_streams(device)
+    mode_id = _lib.SEL[mode] if isinstance(mode, str) else int(mode)
+    check(lib().pbs_attention_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), shp, mode_id, param, scale,
+                                   _ptr(ws), need, _stream(device),
+                                   ctypes.c_void_p(h2d.cuda_stream),
+                                   ctypes.c_void_p(d2h.cuda_stream)), "pbs_attention_host")
+    return o

@@ -330,3 +330,34 @@ def test_fused_unpermute_rejects_output_aliasing_an_input(dev):
     with pytest.raises(pbs.PbsError):
         pbs.attn_fwd(perm["q_perm"], perm["k_perm"], perm["v_perm"], perm["kpos"], perm["kpos"],
                      idx, cnt, B, S, out=perm["q_perm"], unpermute=True)
+
+
+@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128", "odd_items", "d128_b64"])
+def test_host_buffer_path_against_oracle(name, dev):
+    """pbs_attention_host on page-locked host tensors, one KV group at a time
+    with the copies overlapped: against the oracle's pipeline (as the device
+    path), and close to the device path on the same inputs."""
+    w = CASES[name]
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    o_host = pbs.attention_host(qh, kh, vh, w.block, w.segment, w.mode, w.param)
+    torch.cuda.synchronize()
+    assert pbs.device_status() == 0
+    ref = orc.pbs_attention(f64(q), f64(k), f64(v), w.block, w.segment, w.mode, w.param)
+    assert_outputs_close(f64(o_host), ref["o"], name)
+    o_dev = pbs.pbs_attention(qd, kd, vd, w.block, w.segment, w.mode, w.param)
+    assert_outputs_close(f64(o_host), f64(o_dev), "host vs device path")
+
+
+def test_host_buffer_path_many_groups_reuse_both_slots(dev):
+    """Eight KV groups over two batches: every slot is reused several times
+    and each group's output lands at its own place."""
+    w = Workload("groups8", 2, 8, 4, 1024, 128, 128, 256, "topk_frac", 0.5, "uniform", 0.05,
+                 seed=11)
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    o_host = pbs.attention_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), w.block,
+                                w.segment, w.mode, w.param)
+    o_dev = pbs.pbs_attention(qd, kd, vd, w.block, w.segment, w.mode, w.param)
+    torch.cuda.synchronize()
+    assert pbs.device_status() == 0
+    assert_outputs_close(f64(o_host), f64(o_dev), "host vs device path")
