@@ -339,3 +339,59 @@ def dense_causal(q, k, v, scale=None):
 def block_flops(cnt, block, d):
     """Tensor-core work of the forward: 4*B*B*d per kept (head, block) pair."""
     return 4.0 * block * block * d * float(np.asarray(cnt, dtype=np.int64).sum())
+
+
+# --------------------------------------------------------------------------
+# Diagnostics: attention coverage and block-level density
+# (sciencestack.ai Figure 2 caption: the coverage of a selection is the total
+#  attention score its blocks hold; Figure 4: block-level density with and
+#  without permutation; gist.science "Experimentelle Ergebnisse", Sparsity)
+# --------------------------------------------------------------------------
+def block_mass(q, k_perm, kpos, block, scale=None):
+    """Exact attention mass of every (query block, key block) pair.
+
+    Query row i (natural order) attends causally over all n keys: the key in
+    permuted slot p is visible when its original position kpos[p] <= i
+    (kpos None: identity). With the dense softmax probabilities P_ip,
+    mass[b, g, I, J] = (1/B) * sum over rows i of block I and slots p of
+    block J of P_ip. Every (b, g, I) row of mass sums to 1.
+    q: [b, hq, n, d]; k_perm: [b, hkv, n, d]; kpos: [b, hkv, n] or None.
+    Returns [b, hq, nb, nb] fp64.
+    """
+    b, hq, n, d = q.shape
+    hkv = k_perm.shape[1]
+    g_sz = hq // hkv
+    nb = n // block
+    sigma = resolve_scale(scale, d)
+    mass = np.zeros((b, hq, nb, nb))
+    for bi in range(b):
+        for g in range(hq):
+            h = g // g_sz
+            orig = np.arange(n) if kpos is None else kpos[bi, h]
+            logits = sigma * (q[bi, g] @ k_perm[bi, h].T)              # [n, n]
+            visible = orig[None, :] <= np.arange(n)[:, None]
+            p = _softmax_rows(np.where(visible, logits, -np.inf))
+            mass[bi, g] = p.reshape(nb, block, nb, block).sum(axis=(1, 3)) / block
+    return mass
+
+
+def coverage(mass, idx, cnt):
+    """Mass held by each (b, g, I) selection: sum of mass[b, g, I, J] over the
+    first cnt entries J of idx[b, g, I]. Returns [b, hq, nb] fp64."""
+    b, hq, nb, _ = mass.shape
+    out = np.zeros((b, hq, nb))
+    for bi, g, i in np.ndindex(b, hq, nb):
+        out[bi, g, i] = mass[bi, g, i, idx[bi, g, i, :cnt[bi, g, i]]].sum()
+    return out
+
+
+def blocks_for_coverage(mass, target):
+    """Fewest key blocks that hold at least `target` of each row's mass:
+    the blocks in descending mass, counted until their sum reaches target.
+    Returns [b, hq, nb] int64."""
+    b, hq, nb, _ = mass.shape
+    out = np.zeros((b, hq, nb), dtype=np.int64)
+    for bi, g, i in np.ndindex(b, hq, nb):
+        run = np.cumsum(np.sort(mass[bi, g, i])[::-1])
+        out[bi, g, i] = min(nb, int(np.searchsorted(run, target)) + 1)
+    return out

@@ -360,3 +360,84 @@ def test_unpermute_inverts_gather():
     x = rng.standard_normal((2, 3, 32, 4))
     pos = within_segment_perm(rng, 2, 3, 32, 8)
     np.testing.assert_array_equal(orc.unpermute(orc.gather_rows(x, pos), pos), x)
+
+
+# ---------------------------------------------------------------- diagnostics
+def _diag_inputs(seed=4, n=256, block=16, segment=64, hq=2, hkv=1, d=16):
+    g = np.random.default_rng(seed)
+    q = g.standard_normal((1, hq, n, d))
+    k = g.standard_normal((1, hkv, n, d))
+    v = g.standard_normal((1, hkv, n, d))
+    return q, k, v, block, segment
+
+
+def test_block_mass_rows_sum_to_one_and_respect_causality():
+    q, k, _, B, S = _diag_inputs()
+    m = orc.block_mass(q, k, None, B)
+    np.testing.assert_allclose(m.sum(-1), 1.0, atol=1e-12)
+    nb = m.shape[-1]
+    assert np.all(m[..., np.triu_indices(nb, 1)[0], np.triu_indices(nb, 1)[1]] == 0)
+
+
+def test_block_mass_is_attention_probability_mass():
+    # brute force from torch's attention probabilities (V = identity)
+    q, k, _, B, S = _diag_inputs(n=64, block=8, hq=1, d=8)
+    n = q.shape[2]
+    eye = torch.eye(n, dtype=torch.float64)[None, None]
+    probs = sdpa(q, k, eye, causal=True)[0, 0]               # [n, n] = P
+    want = probs.reshape(n // 8, 8, n // 8, 8).sum(axis=(1, 3)) / 8
+    np.testing.assert_allclose(orc.block_mass(q, k, None, 8)[0, 0], want, atol=1e-12)
+
+
+def test_block_mass_permutation_moves_mass_only_inside_segments():
+    # Lemma 3.1: the probabilities do not change, only the blocks they fall in;
+    # a segment's total mass is the same with and without permutation
+    q, k, v, B, S = _diag_inputs()
+    imp = orc.score(q, k, B)
+    perm = orc.permute(imp, k, v, S)
+    m0 = orc.block_mass(q, k, None, B)
+    m1 = orc.block_mass(q, perm["k_perm"], perm["kpos"], B)
+    spb = S // B
+    seg = lambda m: m.reshape(*m.shape[:3], -1, spb).sum(-1)
+    np.testing.assert_allclose(seg(m0), seg(m1), atol=1e-12)
+    assert not np.allclose(m0, m1)
+
+
+def test_coverage_of_all_blocks_is_one_and_of_own_block_is_its_mass():
+    q, k, _, B, S = _diag_inputs()
+    m = orc.block_mass(q, k, None, B)
+    nb = m.shape[-1]
+    idx = np.tile(np.arange(nb), (1, 2, nb, 1)).astype(np.int32)
+    cnt = np.broadcast_to(np.arange(1, nb + 1), (1, 2, nb)).astype(np.int32)
+    np.testing.assert_allclose(orc.coverage(m, idx, cnt), 1.0, atol=1e-12)
+    own = np.broadcast_to(np.arange(nb)[:, None], (1, 2, nb, 1)).astype(np.int32)
+    one = np.ones((1, 2, nb), dtype=np.int32)
+    np.testing.assert_allclose(orc.coverage(m, own, one),
+                               np.diagonal(m, axis1=2, axis2=3), atol=1e-15)
+
+
+def test_blocks_for_coverage_brute_force():
+    q, k, _, B, S = _diag_inputs(n=128, block=16)
+    m = orc.block_mass(q, k, None, B)
+    for target in (0.5, 0.9, 0.975, 1.0 - 1e-9):
+        got = orc.blocks_for_coverage(m, target)
+        for bi, g, i in np.ndindex(*got.shape):
+            row = m[bi, g, i]
+            # fewest blocks of any subset reaching the target, by enumeration
+            nb = len(row)
+            best = min(r for r in range(1, nb + 1)
+                       for c in itertools.combinations(range(nb), r)
+                       if row[list(c)].sum() >= target - 1e-15)
+            assert got[bi, g, i] == best
+
+
+def test_blocks_for_coverage_planted_key():
+    # one key with an overwhelming logit for every query after it: its block
+    # alone holds almost all the mass of every later query block
+    q, k, _, B, S = _diag_inputs(n=128, block=16, hq=1)
+    k[0, 0, 40] = 50.0 * q[0, 0].mean(axis=0) / np.linalg.norm(q[0, 0].mean(axis=0))
+    q[0, 0] += q[0, 0].mean(axis=0)
+    m = orc.block_mass(q, k, None, B)
+    got = orc.blocks_for_coverage(m, 0.5)
+    assert np.all(got[0, 0, 3:] == 1)
+    assert np.all(m[0, 0, 3:, 2] > 0.5)
