@@ -12,6 +12,8 @@
  *   pbs_unpermute      inverse permutation of the output rows
  *   pbs_attn_fwd_unpermute  the last two fused: rows written in place
  *   pbs_attention_host the whole path on host buffers, copies overlapped
+ *   pbs_block_mass, pbs_coverage  diagnostics: attention coverage and
+ *                      block-level density
  *
  * Conventions shared by every call
  * --------------------------------
@@ -286,6 +288,43 @@ pbs_status pbs_attention_host(const void *q, const void *k, const void *v,
                               float scale, void *ws, size_t ws_bytes,
                               pbs_stream_t compute, pbs_stream_t h2d,
                               pbs_stream_t d2h);
+
+/*
+ * pbs_block_mass - diagnostics: the exact attention mass of every (query
+ * block, key block) pair. Source: sciencestack.ai Figure 2 caption (the
+ * attention coverage of a selection is the total attention score its blocks
+ * hold) and Figure 4 (block-level density with and without permutation).
+ *
+ * Query row i (natural order) attends over all n keys: the key in permuted
+ * slot p is visible when kpos[p] <= i (kpos NULL: the identity, i.e. the
+ * unpermuted sequence). With the dense softmax probabilities P_ip,
+ * mass[b, g, I, J] = (1/B) sum over rows i of block I and slots p of block J
+ * of P_ip; every (b, g, I) row sums to 1 and entries J past the admissible
+ * blocks of I are 0. Two passes over the admissible keys on the tensor cores.
+ *
+ *   q       [batch, hq, n, d] bf16 (natural order)
+ *   k_perm  [batch, hkv, n, d] bf16; kpos [batch, hkv, n] int32 or NULL
+ *   mass    [batch, hq, nb, nb] fp32, written
+ * Supported: block = 128, hq / hkv <= 4 (else PBS_ERR_UNSUPPORTED).
+ */
+pbs_status pbs_block_mass(const void *q, const void *k_perm, const int32_t *kpos,
+                          float *mass, pbs_shape s, float scale, pbs_stream_t st);
+
+/*
+ * pbs_coverage - diagnostics on a block mass (as from pbs_block_mass), per
+ * (b, g, I) row: the mass its list of kept blocks holds, and the fewest
+ * blocks that hold at least `target` of the row's mass (the blocks in
+ * descending mass, counted until their sum reaches the target; nb when the
+ * row's total is below it). Sums in fp64, in a fixed order.
+ *
+ *   mass             [batch, hq, nb, nb] fp32
+ *   blk_idx, blk_cnt as written by pbs_select_blocks; needed for coverage
+ *   coverage         [batch, hq, nb] fp32, or NULL
+ *   blocks_needed    [batch, hq, nb] int32, or NULL; target in (0, 1]
+ */
+pbs_status pbs_coverage(const float *mass, const int32_t *blk_idx,
+                        const int32_t *blk_cnt, double target, float *coverage,
+                        int32_t *blocks_needed, pbs_shape s, pbs_stream_t st);
 
 /*
  * Synchronises `st`, returns in *code the current device's error word

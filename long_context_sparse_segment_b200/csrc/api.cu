@@ -349,6 +349,36 @@ pbs_status pbs_attention_host(const void *q, const void *k, const void *v, void 
   return cuda_status(e);
 }
 
+pbs_status pbs_block_mass(const void *q, const void *k_perm, const int32_t *kpos, float *mass,
+                          pbs_shape s, float scale, pbs_stream_t st) {
+  Dims dm;
+  pbs_status r = check_shape(s, &dm);
+  if (r != PBS_OK) return r;
+  if (empty(dm)) return PBS_OK;
+  if (!q || !k_perm || !mass || !aligned16(q) || !aligned16(k_perm) || (kpos && !aligned16(kpos)) ||
+      ((uintptr_t)mass & 3u))
+    return PBS_ERR_INVALID_ARG;
+  if (!mass_supported(dm)) return PBS_ERR_UNSUPPORTED;
+  const float sigma = (float)resolve_sigma(scale, dm.d);
+  return cuda_status(
+      launch_block_mass(dm, q, k_perm, kpos, mass, sigma, error_word(), (cudaStream_t)st));
+}
+
+pbs_status pbs_coverage(const float *mass, const int32_t *blk_idx, const int32_t *blk_cnt,
+                        double target, float *coverage, int32_t *blocks_needed, pbs_shape s,
+                        pbs_stream_t st) {
+  Dims dm;
+  pbs_status r = check_shape(s, &dm);
+  if (r != PBS_OK) return r;
+  if (empty(dm)) return PBS_OK;
+  if (!mass || ((uintptr_t)mass & 3u)) return PBS_ERR_INVALID_ARG;
+  if (coverage && (!blk_idx || !blk_cnt)) return PBS_ERR_INVALID_ARG;
+  if (blocks_needed && !(target > 0.0 && target <= 1.0)) return PBS_ERR_INVALID_ARG;
+  const int rows = dm.b * dm.hq * dm.nb;
+  return cuda_status(launch_coverage(mass, coverage ? blk_idx : nullptr, blk_cnt, target, rows,
+                                     dm.nb, coverage, blocks_needed, (cudaStream_t)st));
+}
+
 pbs_status pbs_get_device_status(pbs_stream_t st, int *code, int *detail) {
   if (!code) return PBS_ERR_INVALID_ARG;
   if (cudaStreamSynchronize((cudaStream_t)st) != cudaSuccess) return PBS_ERR_CUDA;

@@ -70,6 +70,15 @@ cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const
                             const int32_t *cnt, void *out, float *lse, float sigma, int *err,
                             bool scatter, cudaStream_t st);
 
+// diagnostics: block attention mass (tcgen05, B = 128, G <= 4), and per row
+// the coverage of a list and the fewest blocks for a target coverage
+bool mass_supported(const Dims &dm);
+cudaError_t launch_block_mass(const Dims &dm, const void *q, const void *kp, const int32_t *kpos,
+                              float *mass, float sigma, int *err, cudaStream_t st);
+cudaError_t launch_coverage(const float *mass, const int32_t *idx, const int32_t *cnt,
+                            double target, int rows, int nb, float *cov, int32_t *kmin,
+                            cudaStream_t st);
+
 // out[qpos[p]] = out_perm[p]
 cudaError_t launch_unpermute(const Dims &dm, const void *op, const int32_t *qpos, void *out,
                              int *err, cudaStream_t st);
