@@ -70,3 +70,45 @@ def report(q, k, v, block, segment, mode, param, target=0.975, scale=0.0):
     }
     out["ideal_block_reduction"] = 1.0 - out["ideal_density_perm"] / out["ideal_density_noperm"]
     return out
+
+
+def _main():
+    import argparse
+    import json
+
+    from .workloads import WORKLOADS, make_inputs
+
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--config", default="llama32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--target", type=float, default=0.975)
+    ap.add_argument("--strength", type=float, default=None,
+                    help="planted-key strength (K += strength * u) instead of the workload's")
+    args = ap.parse_args()
+    w = WORKLOADS[args.config]
+    if args.strength is not None:
+        w = w.with_(strength=args.strength)
+    dev = torch.device("cuda", 0)
+    q, k, v, _ = make_inputs(w, dev)
+    out = {"workload": w.name, "strength": w.strength, **report(q, k, v, w.block, w.segment, w.mode, w.param,
+                                       args.target)}
+    # time the block-mass pass on the permuted keys (tensor work: two QK
+    # products per admissible (head, key block) pair)
+    res = ops.pbs_attention(q, k, v, w.block, w.segment, w.mode, w.param, keep=True)
+    block_mass(q, res["k_perm"], res["kpos"], w.block, w.segment)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    block_mass(q, res["k_perm"], res["kpos"], w.block, w.segment)
+    e1.record()
+    torch.cuda.synchronize()
+    nb, spb = w.n // w.block, w.segment // w.block
+    pairs = w.batch * w.hq * sum(min(nb, (i // spb + 1) * spb) for i in range(nb))
+    ms = e0.elapsed_time(e1)
+    out["block_mass_ms"] = round(ms, 3)
+    out["block_mass_tflops"] = round(2 * 2.0 * w.block * w.block * w.d * pairs / ms / 1e9, 1)
+    out["status"] = ops.device_status()
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    _main()

@@ -44,6 +44,7 @@ class Workload:
     layers: int = 1
     seed: int = 0
     burst: int = 16
+    strength: float = 3.0  # planted keys get K += strength * u
 
     @property
     def group(self) -> int:
@@ -122,7 +123,7 @@ def make_inputs(w: Workload, device="cpu", layer: int = 0, seed: int | None = No
                     dtype=torch.float32)
     u = u / u.norm(dim=-1, keepdim=True)
     sal = salient_mask(w, gen, device)
-    k += 3.0 * sal.unsqueeze(-1).float() * u.unsqueeze(2)
+    k += w.strength * sal.unsqueeze(-1).float() * u.unsqueeze(2)
     q += u.repeat_interleave(w.group, dim=1).unsqueeze(2)
     out = (q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16))
     del q, k, v
