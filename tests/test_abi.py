@@ -110,3 +110,53 @@ def test_workspace_sizes_grow_with_the_problem(lib):
     b = pbs.workspace_bytes(shape(n=2048), _lib.OP_SELECT)
     assert b == 2 * a > 0
     assert pbs.workspace_bytes(shape(), _lib.OP_ATTN) == 0
+
+
+def test_fused_forward_rejects_output_aliasing_an_input(lib):
+    s = shape()
+    fake = ctypes.c_void_p(1 << 20)
+    other = ctypes.c_void_p(1 << 24)
+    for out in (fake,):
+        assert lib.pbs_attn_fwd_unpermute(fake, other, other, None, other, other, other, out,
+                                          None, s, 0.0, None) == _lib.ERR_INVALID_ARG
+
+
+def test_host_path_arguments(lib):
+    s = shape()
+    fake = ctypes.c_void_p(1 << 20)
+    ws = pbs.workspace_bytes(s, _lib.OP_HOST_PATH)
+    assert ws > 0
+    call = lambda *a: lib.pbs_attention_host(*a)
+    for mode, param in ((0, 0.0), (1, 1.5), (9, 0.5)):
+        assert call(fake, fake, fake, fake, s, mode, param, 0.0, fake, ws, None, None,
+                    None) == _lib.ERR_INVALID_ARG
+    assert call(None, fake, fake, fake, s, 0, 0.9, 0.0, fake, ws, None, None,
+                None) == _lib.ERR_INVALID_ARG
+    assert call(fake, fake, fake, fake, s, 0, 0.9, 0.0, fake, ws - 1, None, None,
+                None) == _lib.ERR_WORKSPACE
+    # a KV group of 16 query heads x B = 128 probe rows exceeds the scoring kernels
+    big = shape(hq=16, hkv=1)
+    assert call(fake, fake, fake, fake, big, 0, 0.9, 0.0, fake, 1 << 40, None, None,
+                None) == _lib.ERR_UNSUPPORTED
+    assert call(None, None, None, None, shape(n=0), 0, 0.9, 0.0, None, 0, None, None, None) == 0
+    # two slots of one KV group's buffers: the size grows with n, not with the group count
+    assert pbs.workspace_bytes(shape(n=2048), _lib.OP_HOST_PATH) > ws
+    assert pbs.workspace_bytes(shape(batch=4), _lib.OP_HOST_PATH) == ws
+
+
+def test_diagnostics_arguments(lib):
+    s = shape()
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    assert lib.pbs_block_mass(fake, fake, None, fake, shape(block=64), 0.0,
+                              None) == _lib.ERR_UNSUPPORTED
+    assert lib.pbs_block_mass(fake, fake, None, fake, shape(hq=16, hkv=2), 0.0,
+                              None) == _lib.ERR_UNSUPPORTED
+    assert lib.pbs_block_mass(None, fake, None, fake, s, 0.0, None) == _lib.ERR_INVALID_ARG
+    assert lib.pbs_block_mass(fake, fake, None, odd, s, 0.0, None) == _lib.ERR_INVALID_ARG
+    # coverage needs the lists; the target must lie in (0, 1]
+    assert lib.pbs_coverage(fake, None, None, ctypes.c_double(0.9), fake, None, s,
+                            None) == _lib.ERR_INVALID_ARG
+    for t in (0.0, 1.5):
+        assert lib.pbs_coverage(fake, None, None, ctypes.c_double(t), None, fake, s,
+                                None) == _lib.ERR_INVALID_ARG
