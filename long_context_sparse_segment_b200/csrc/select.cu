@@ -69,6 +69,34 @@ __device__ __forceinline__ double warp_max_d(double v) {
   return v;
 }
 
+// The bits every key[0 .. cnt) shares: on return *pre holds them (the other
+// bits 0) and the result is the index of the highest bit at which two keys
+// differ, or -1 when all are equal (then *pre is the common key).
+__device__ __forceinline__ int common_prefix(const unsigned long long *key, int cnt, int lane,
+                                             unsigned long long *pre) {
+  unsigned long long mn = ~0ull, mx = 0ull;
+  for (int J = lane; J < cnt; J += 32) {
+    const unsigned long long k = key[J];
+    mn = k < mn ? k : mn;
+    mx = k > mx ? k : mx;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, mn, o);
+    const unsigned long long b = __shfl_xor_sync(0xffffffffu, mx, o);
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+  const unsigned long long diff = mn ^ mx;
+  if (diff == 0) {
+    *pre = mx;
+    return -1;
+  }
+  const int top = 63 - __clzll((long long)diff);
+  *pre = top == 63 ? 0ull : mx & ~((2ull << top) - 1);
+  return top;
+}
+
 // D[8x8] += A[8x4] * B[4x8] in fp64: lane t holds A[t/4][t%4], B[t%4][t/4],
 // D[t/4][2(t%4)] and D[t/4][2(t%4)+1].
 __device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
@@ -174,10 +202,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the keys that share the digits found so far, count each value of
         // the next digit, and take the digit at which the count from the top
         // reaches the number still needed.
+        // The bits all keys share are skipped: they would send every key to
+        // one histogram bin.
         unsigned *hist = hists + w * 256;
-        unsigned long long pre = 0, pmask = 0;
+        unsigned long long pre = 0;
+        const int top = common_prefix(key, f0, lane, &pre);
         int need = t;
-        for (int shift = 56; shift >= 0; shift -= 8) {
+        const int first = top < 0 ? -8 : (top / 8) * 8;  // the byte holding the top bit
+        unsigned long long pmask = first + 8 >= 64 ? 0ull : ~((1ull << (first + 8)) - 1);
+        pre &= pmask;  // the shared bits inside the first byte come with its digit
+        for (int shift = first; shift >= 0; shift -= 8) {
           for (int d = lane; d < 256; d += 32) hist[d] = 0;
           __syncwarp();
           for (int J = lane; J < f0; J += 32) {
@@ -218,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pmask |= 255ull << shift;
           __syncwarp();
         }
-        kcut = pre;
+        kcut = pre;  // all keys equal (top < 0): the common key
         tie_take = need;  // keys equal to the cut that are still taken
       }
     } else {
@@ -247,8 +281,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (mass_ge(0ull) < tau) {
           all_earlier = true;  // the mass never reaches tau: every block
         } else {
-          unsigned long long k = 0;  // largest value whose mass still reaches tau
-          for (int bit = 63; bit >= 0; --bit) {
+          // largest value whose mass still reaches tau; it lies between the
+          // smallest and largest key, so the bits they share are fixed
+          unsigned long long k = 0;
+          const int top = common_prefix(key, f0, lane, &k);
+          for (int bit = top; bit >= 0; --bit) {
             const unsigned long long cand = k | (1ull << bit);
             if (mass_ge(cand) >= tau) k = cand;
           }
