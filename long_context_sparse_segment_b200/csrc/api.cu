@@ -199,20 +199,23 @@ pbs_status pbs_select_blocks(const void *q_or_qperm, const void *k_perm, const d
   }
   int *err = error_word();
   cudaStream_t cs = (cudaStream_t)st;
+  // workspace (scored modes only): qsum | [ksum when not given] | scratch
   double *qsum = (double *)ws;
   const double *ksum = kbar_sum;
+  uint8_t *scratch = scored ? (uint8_t *)ws + select_qsum_bytes(dm) : nullptr;
   if (scored) {
     cudaError_t e = launch_blocksum(dm, dm.b * dm.hq, q_or_qperm, qsum, cs);
     if (e != cudaSuccess) return PBS_ERR_CUDA;
     if (!kbar_sum) {
-      double *kbuf = qsum + (size_t)dm.b * dm.hq * dm.nb * dm.d;
+      double *kbuf = (double *)scratch;
       e = launch_blocksum(dm, dm.b * dm.hkv, k_perm, kbuf, cs);
       if (e != cudaSuccess) return PBS_ERR_CUDA;
       ksum = kbuf;
+      scratch += (size_t)dm.b * dm.hkv * dm.nb * dm.d * 8;
     }
   }
   return cuda_status(launch_select(dm, qsum, ksum, mode, param, resolve_sigma(scale, dm.d),
-                                   blk_idx, blk_cnt, blk_mask, err, cs));
+                                   blk_idx, blk_cnt, blk_mask, scratch, err, cs));
 }
 
 namespace {
@@ -331,7 +334,8 @@ pbs_status pbs_attention_host(const void *q, const void *k, const void *v, void 
       e = launch_gather(g, sl.kpos, sl.k, sl.v, nullptr, sl.kp, sl.vp, nullptr, sl.kbar, err, cs);
     if (e == cudaSuccess && scored) e = launch_blocksum(g, g.hq, sl.q, sl.qsum, cs);
     if (e == cudaSuccess)
-      e = launch_select(g, sl.qsum, sl.kbar, mode, param, sigma_d, sl.idx, sl.cnt, nullptr, err, cs);
+      e = launch_select(g, sl.qsum, sl.kbar, mode, param, sigma_d, sl.idx, sl.cnt, nullptr,
+                        (uint8_t *)sl.qsum + select_qsum_bytes(g), err, cs);
     if (e == cudaSuccess)
       e = launch_attn(g, sl.q, sl.kp, sl.vp, sl.kpos, nullptr, sl.idx, sl.cnt, sl.o, nullptr,
                       sigma_f, err, false, cs);

@@ -39,10 +39,14 @@ cudaError_t launch_blocksum(const Dims &dm, int heads, const void *x, double *ou
                             cudaStream_t st);
 
 // block lists from pooled sums
+// workspace: pooled query sums [+ pooled key sums] + scratch (score keys and
+// softmax weights per (batch, query head, query block, key block))
 size_t select_ws_bytes(const Dims &dm, bool need_kbar);
+size_t select_qsum_bytes(const Dims &dm);
+size_t select_scratch_bytes(const Dims &dm);
 cudaError_t launch_select(const Dims &dm, const double *qsum, const double *ksum, int mode,
                           float param, double sigma, int32_t *idx, int32_t *cnt,
-                          uint8_t *mask, int *err, cudaStream_t st);
+                          uint8_t *mask, void *scratch, int *err, cudaStream_t st);
 
 // block-sparse forward; with `scatter` each output row is written at its
 // query's original position (qpos) instead of its place in the given order

@@ -8,21 +8,25 @@
 // blocks, at least one).
 //
 // All decisions are taken in fp64 from fp64 block sums (exact for bf16
-// rows). One CTA per (batch, query head, up to 8 consecutive query blocks):
-//   scores a_IJ = sigma * qbar_I . kbar_J on the fp64 tensor cores
-//     (mma.sync m8n8k4: the CTA's rows are M = 8, each warp owns 8 key
-//     blocks of a 64-block chunk staged in shared memory);
-//   then one warp per query block decides, without sorting:
+// rows). Two kernels:
+//   scores: a_IJ = sigma * qbar_I . kbar_J for every admissible (I, J) on the
+//     fp64 tensor cores (mma.sync m8n8k4, 64 x 64 tiles of query blocks by
+//     key blocks, d staged once in shared memory), written to the workspace
+//     as 64-bit order keys: every pooled key block is read once per tile
+//     instead of once per query block;
+//   selection: one warp per query block decides, without sorting, reading
+//     its row of keys from the workspace (L1/L2):
 //   TOPK_FRAC: k = max(1, floor(f * (I + 1))); the t = max(0, k - own)
 //     earlier-segment blocks of largest score (ties: lower J) are found by
-//     a radix select over the 64-bit order keys of the scores (eight rounds
-//     of 8-bit digit histograms: the t-th largest key and how many of the
-//     keys equal to it are taken);
-//   THRESHOLD: softmax over the admissible blocks; bisection finds the
-//     largest score s such that the own-segment mass plus the mass of the
-//     earlier blocks scoring >= s reaches tau; blocks scoring above s are
-//     kept and blocks tied at s are added in ascending J until it does. This
-//     is the set the descending walk of the definition stops at.
+//     a radix select over the order keys (8-bit digit histograms from the
+//     first byte in which the row's keys differ: the t-th largest key and
+//     how many of the keys equal to it are taken);
+//   THRESHOLD: softmax over the admissible blocks (weights to the
+//     workspace); bisection finds the largest score s such that the
+//     own-segment mass plus the mass of the earlier blocks scoring >= s
+//     reaches tau; blocks scoring above s are kept and blocks tied at s are
+//     added in ascending J until it does. This is the set the descending
+//     walk of the definition stops at.
 // then the warp compacts the kept flags into the ascending list. Masses are
 // summed in a fixed order, so results are deterministic.
 #include <math.h>
@@ -33,25 +37,15 @@
 namespace pbs {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kChunk = 64;       // key blocks per staged chunk: 8 warps x 8
-constexpr int kPad = 132;        // doubles per staged row: conflict-free B reads
-constexpr size_t kSmemBudget = 220 * 1024;
+constexpr int kThreads = 256;  // selection: 8 warps, one query block each
+constexpr int kTile = 64;      // score tiles: 64 query blocks x 64 key blocks
+constexpr int kPad = 4;        // doubles of padding per staged row (bank spread)
 
 constexpr int kWarps = kThreads / 32;
 
-// Score keys are stored with a row stride of nb + 1 words, so that the
-// eight rows of one tensor-core result land in different banks.
-size_t sel_smem(int rows, int nb) {
-  return (size_t)kChunk * kPad * 8 + (size_t)rows * (nb + 1) * 8 + (size_t)rows * nb * (8 + 1) +
-         kWarps * 256 * 4 + 64;
-}
-
-int sel_rows(int nb) {
-  int r = 8;
-  while (r > 1 && sel_smem(r, nb) > kSmemBudget) r >>= 1;
-  return r;
-}
+// selection shared memory: per warp, the kept flags of its row and a digit
+// histogram
+size_t sel_smem(int nb) { return (size_t)kWarps * ((size_t)nb + 256 * 4) + 64; }
 
 __device__ __forceinline__ double f64_from_order_key(unsigned long long u) {
   return __longlong_as_double(
@@ -105,86 +99,93 @@ __device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
                : "d"(a), "d"(b));
 }
 
+// Scores of one 64 x 64 tile of (query block I, key block J) pairs of one
+// (batch, query head): a_IJ = sigma * qbar_I . kbar_J with the block means
+// qbar = qsum / B, kbar = ksum / B, as 64-bit order keys into
+// keys[bg][I][J] for the admissible J (segment of J <= segment of I).
+// 8 warps as 2 x 4: a warp owns 32 query blocks x 16 key blocks, i.e. 4 x 2
+// m8n8k4 products per 4-wide step of d.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    select_kernel(const double *__restrict__ qsum, const double *__restrict__ ksum, Dims dm,
-                  int mode, float param, double sigma, int rows, int32_t *__restrict__ idx_out,
+    scores_kernel(const double *__restrict__ qsum, const double *__restrict__ ksum, Dims dm,
+                  double sigma, unsigned long long *__restrict__ keys) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int LD = D + kPad;
+  double *As = reinterpret_cast<double *>(smem);  // [kTile][LD] query block means
+  double *Bs = As + kTile * LD;                   // [kTile][LD] key block means
+  const int nb = dm.nb;
+  const int bg = blockIdx.z, b = bg / dm.hq, g = bg % dm.hq;
+  const int kv = b * dm.hkv + g / dm.G;
+  const int R0 = blockIdx.y * kTile, C0 = blockIdx.x * kTile;
+  const int last = min(nb, R0 + kTile) - 1;
+  if (C0 >= min(nb, (last / dm.spb + 1) * dm.spb)) return;  // nothing admissible here
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const double inv_b = 1.0 / (double)dm.B;  // a power of two: exact
+  for (int e = tid; e < kTile * D; e += kThreads) {
+    const int r = e / D, c = e % D;
+    As[r * LD + c] = R0 + r < nb ? qsum[((size_t)bg * nb + R0 + r) * D + c] * inv_b : 0.0;
+    Bs[r * LD + c] = C0 + r < nb ? ksum[((size_t)kv * nb + C0 + r) * D + c] * inv_b : 0.0;
+  }
+  __syncthreads();
+  const int wr = (w >> 2) * 32, wc = (w & 3) * 16;
+  double acc[4][2][2];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = 0.0;
+  const double *ap = As + (wr + (lane >> 2)) * LD + (lane & 3);
+  const double *bp = Bs + (wc + (lane >> 2)) * LD + (lane & 3);
+#pragma unroll 4
+  for (int k = 0; k < D; k += 4) {
+    double af[4], bf[2];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) af[mt] = ap[mt * 8 * LD + k];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) bf[nt] = bp[nt * 8 * LD + k];
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) dmma_8x8x4(acc[mt][nt], af[mt], bf[nt]);
+  }
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const int I = R0 + wr + mt * 8 + (lane >> 2);
+    if (I >= nb) continue;
+    const int adm = min(nb, (I / dm.spb + 1) * dm.spb);
+    unsigned long long *row = keys + ((size_t)bg * nb + I) * nb;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int J = C0 + wc + nt * 8 + 2 * (lane & 3) + u;
+        if (J < adm) row[J] = f64_order_key(sigma * acc[mt][nt][u]);
+      }
+  }
+}
+
+// One warp per (batch, query head, query block): the kept list from the
+// row's score keys (and, for THRESHOLD, softmax weights written next to
+// them in `pis`).
+__global__ void __launch_bounds__(kThreads)
+    select_kernel(const unsigned long long *__restrict__ keys, double *__restrict__ pis_all,
+                  Dims dm, int mode, float param, int32_t *__restrict__ idx_out,
                   int32_t *__restrict__ cnt_out, uint8_t *__restrict__ mask_out) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int nb = dm.nb;
-  double *kb = reinterpret_cast<double *>(smem);  // [kChunk][kPad]
-  unsigned long long *keys =
-      reinterpret_cast<unsigned long long *>(kb + kChunk * kPad);  // [rows][nb + 1]
-  double *pis = reinterpret_cast<double *>(keys + (size_t)rows * (nb + 1));  // [rows][nb]
-  unsigned *hists = reinterpret_cast<unsigned *>(pis + (size_t)rows * nb);  // [kWarps][256]
-  unsigned char *flags = reinterpret_cast<unsigned char *>(hists + kWarps * 256);
-
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int bg = blockIdx.y, b = bg / dm.hq, g = bg % dm.hq;
-  const int kv = b * dm.hkv + g / dm.G;
-  const int I0 = blockIdx.x * rows;
-  const int nrows = min(rows, nb - I0);
+  const long long rowid = (long long)blockIdx.x * kWarps + w;
+  if (rowid >= (long long)dm.b * dm.hq * nb) return;  // whole warp; no block barrier follows
+  unsigned *hists = reinterpret_cast<unsigned *>(smem);  // [kWarps][256]
+  unsigned char *flag = reinterpret_cast<unsigned char *>(hists + kWarps * 256) + (size_t)w * nb;
+  const int bg = (int)(rowid / nb);
   const bool scored = mode == PBS_SEL_THRESHOLD || mode == PBS_SEL_TOPK_FRAC;
-  const double inv_b = 1.0 / (double)dm.B;
 
-  if (scored) {
-    // A fragments: this lane's element of row t/4 for every 4-wide step of d
-    const int ar = lane >> 2;
-    double a[D / 4];
-#pragma unroll
-    for (int k = 0; k < D / 4; ++k)
-      a[k] = ar < nrows ? qsum[((size_t)bg * nb + I0 + ar) * D + 4 * k + (lane & 3)] * inv_b : 0.0;
-    const int last = I0 + nrows - 1;
-    const int max_adm = min(nb, (last / dm.spb + 1) * dm.spb);
-    const double *kbase = ksum + (size_t)kv * nb * D;
-    constexpr int NL = kChunk * D / kThreads;
-    double pre[NL];
-    auto fetch = [&](int c0) {
-#pragma unroll
-      for (int k = 0; k < NL; ++k) {
-        const int e = tid + k * kThreads, J = c0 + e / D;
-        pre[k] = J < nb ? kbase[(size_t)J * D + e % D] : 0.0;
-      }
-    };
-    fetch(0);
-    for (int c0 = 0; c0 < max_adm; c0 += kChunk) {
-      __syncthreads();
-#pragma unroll
-      for (int k = 0; k < NL; ++k) {
-        const int e = tid + k * kThreads;
-        kb[(e / D) * kPad + e % D] = pre[k] * inv_b;
-      }
-      __syncthreads();
-      if (c0 + kChunk < max_adm) fetch(c0 + kChunk);
-      // four independent accumulation chains over d, added in a fixed order
-      double acc4[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
-      const double *brow = kb + (w * 8 + (lane >> 2)) * kPad + (lane & 3);
-#pragma unroll
-      for (int k = 0; k < D / 4; ++k) dmma_8x8x4(acc4[k & 3], a[k], brow[4 * k]);
-      double acc[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) acc[u] = (acc4[0][u] + acc4[1][u]) + (acc4[2][u] + acc4[3][u]);
-      if (ar < nrows) {
-        const int I = I0 + ar;
-        const int adm = min(nb, (I / dm.spb + 1) * dm.spb);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int J = c0 + w * 8 + 2 * (lane & 3) + u;
-          if (J < adm) keys[(size_t)ar * (nb + 1) + J] = f64_order_key(sigma * acc[u]);
-        }
-      }
-    }
-  }
-  __syncthreads();
-  if (w >= nrows) return;  // whole warp, after the last block-wide barrier
-
-  const int I = I0 + w;
+  const int I = (int)(rowid % nb);
   const int seg = I / dm.spb;
   const int f0 = seg * dm.spb;  // own segment: [f0, adm); earlier blocks: [0, f0)
   const int adm = min(nb, f0 + dm.spb);
-  const unsigned long long *key = keys + (size_t)w * (nb + 1);
-  double *pi = pis + (size_t)w * nb;
-  unsigned char *flag = flags + (size_t)w * nb;
+  const unsigned long long *key = keys + (size_t)rowid * nb;
+  double *pi = pis_all + (size_t)rowid * nb;
 
   // Selected earlier blocks: key > kcut, plus `tie_take` of those with
   // key == kcut in ascending J.
@@ -351,24 +352,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+// Workspace: the pooled query sums, [the pooled key sums,] then the score
+// keys and the softmax weights of every (batch, query head, query block,
+// key block).
+size_t select_qsum_bytes(const Dims &dm) { return (size_t)dm.b * dm.hq * dm.nb * dm.d * 8; }
+
+size_t select_scratch_bytes(const Dims &dm) { return 2 * (size_t)dm.b * dm.hq * dm.nb * dm.nb * 8; }
+
 size_t select_ws_bytes(const Dims &dm, bool need_kbar) {
-  size_t q = (size_t)dm.b * dm.hq * dm.nb * dm.d * sizeof(double);
-  size_t k = need_kbar ? (size_t)dm.b * dm.hkv * dm.nb * dm.d * sizeof(double) : 0;
-  return q + k;
+  const size_t k = need_kbar ? (size_t)dm.b * dm.hkv * dm.nb * dm.d * 8 : 0;
+  return select_qsum_bytes(dm) + k + select_scratch_bytes(dm);
 }
 
 cudaError_t launch_select(const Dims &dm, const double *qsum, const double *ksum, int mode,
                           float param, double sigma, int32_t *idx, int32_t *cnt, uint8_t *mask,
-                          int *err, cudaStream_t st) {
+                          void *scratch, int *err, cudaStream_t st) {
   (void)err;
-  const int rows = sel_rows(dm.nb);
-  const size_t smem = sel_smem(rows, dm.nb);
+  const bool scored = mode == PBS_SEL_THRESHOLD || mode == PBS_SEL_TOPK_FRAC;
+  unsigned long long *keys = reinterpret_cast<unsigned long long *>(scratch);
+  double *pis = reinterpret_cast<double *>(keys + (size_t)dm.b * dm.hq * dm.nb * dm.nb);
+  cudaError_t e;
+  if (scored) {
+    auto sk = dm.d == 64 ? scores_kernel<64> : scores_kernel<128>;
+    const size_t ssm = (size_t)2 * kTile * (dm.d + kPad) * 8;
+    e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
+    if (e != cudaSuccess) return e;
+    const int tiles = (dm.nb + kTile - 1) / kTile;
+    sk<<<dim3(tiles, tiles, dm.b * dm.hq), kThreads, ssm, st>>>(qsum, ksum, dm, sigma, keys);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const size_t smem = sel_smem(dm.nb);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  auto kern = dm.d == 64 ? select_kernel<64> : select_kernel<128>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((dm.nb + rows - 1) / rows, dm.b * dm.hq);
-  kern<<<grid, kThreads, smem, st>>>(qsum, ksum, dm, mode, param, sigma, rows, idx, cnt, mask);
+  const long long rows = (long long)dm.b * dm.hq * dm.nb;
+  select_kernel<<<(unsigned)((rows + kWarps - 1) / kWarps), kThreads, smem, st>>>(
+      keys, pis, dm, mode, param, idx, cnt, mask);
   return cudaGetLastError();
 }
 

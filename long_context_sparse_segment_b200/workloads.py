@@ -71,6 +71,12 @@ WORKLOADS = {
     # 128K, fixed top-k of 25% of the causal key blocks per query block.
     "llama128k": Workload("llama128k", 1, 32, 8, 131072, 128, 128, 4096,
                           "topk_frac", 0.25, "per_segment", 0.02),
+    # Longer contexts with the 128K recipe (the pages name 256K and 512K as
+    # the lengths of their largest speedups, without a selection setting).
+    "llama256k": Workload("llama256k", 1, 32, 8, 262144, 128, 128, 4096,
+                          "topk_frac", 0.25, "per_segment", 0.02),
+    "llama512k": Workload("llama512k", 1, 32, 8, 524288, 128, 128, 4096,
+                          "topk_frac", 0.25, "per_segment", 0.02),
     # 32 independent layers at 64K, batch 2; layer l is seeded with l.
     "stack64k": Workload("stack64k", 2, 32, 8, 65536, 128, 128, 2048,
                          "threshold", 0.9, "per_segment", 0.02, layers=32),

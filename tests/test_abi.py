@@ -106,9 +106,12 @@ def test_empty_calls_launch_nothing(lib):
 
 
 def test_workspace_sizes_grow_with_the_problem(lib):
-    a = pbs.workspace_bytes(shape(), _lib.OP_SELECT)
-    b = pbs.workspace_bytes(shape(n=2048), _lib.OP_SELECT)
-    assert b == 2 * a > 0
+    # selection: pooled query and key sums (fp64, per block), then the score
+    # keys and softmax weights of every (query head, query block, key block)
+    for n in (1024, 2048):
+        nb = n // GOOD["block"]
+        want = 8 * nb * GOOD["d"] * (GOOD["hq"] + GOOD["hkv"]) + 2 * 8 * GOOD["hq"] * nb * nb
+        assert pbs.workspace_bytes(shape(n=n), _lib.OP_SELECT) == want
     assert pbs.workspace_bytes(shape(), _lib.OP_ATTN) == 0
 
 
