@@ -183,6 +183,9 @@ pbs_status pbs_permute(const float *imp, const void *k, const void *v,
  *   blk_cnt     [batch, hq, n/B] int32, written
  *   blk_mask    [batch, hq, n/B, n/B] uint8 (1 = kept), written if non-NULL
  *   ws          device workspace of pbs_workspace_bytes(s, PBS_OP_SELECT)
+ *               bytes: the pooled sums and the score of every admissible
+ *               (query block, key block) pair; ALL and DENSE_CAUSAL do not
+ *               use it (NULL accepted)
  */
 pbs_status pbs_select_blocks(const void *q_or_qperm, const void *k_perm,
                              const double *kbar_sum, pbs_shape s, int mode,
