@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--config", default="llama128k", choices=sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: every rank runs the whole workload (weak scaling), or "
+                         "the KV groups of one workload are split over the ranks (strong)")
     ap.add_argument("--profile", action="store_true",
                     help="time the steps only (no dense, end-to-end or CPU legs), for ncu")
     return ap.parse_args()
@@ -68,6 +71,17 @@ RANK_SEED_STRIDE = 1000  # rank r draws its replica's inputs with seed + 1000 r
 
 def rank_seed_offset(rank):
     return RANK_SEED_STRIDE * rank
+
+
+def shard_heads(w, rank, world):
+    """The rank's share of one sequence when the KV groups are split over the
+    ranks (the path is independent per KV group, so no data crosses ranks):
+    KV heads [rank * hkv / world, (rank + 1) * hkv / world) with their query
+    heads. Returns (workload of the share, first KV head)."""
+    if w.hkv % world:
+        raise ValueError(f"{w.hkv} KV heads do not split over {world} ranks")
+    per = w.hkv // world
+    return w.with_(hkv=per, hq=per * w.group), rank * per
 
 
 def job_throughput(flops_rank, ms_rank, dist=None, device="cpu"):
@@ -244,7 +258,15 @@ def gpu_arm(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     w = WORKLOADS[args.config]
-    layers = [Layer(w, dev, l, seed_offset=rank_seed_offset(rank)) for l in range(w.layers)]
+    sharded = args.shard == "heads" and world > 1
+    w_full = w
+    if sharded:
+        # one sequence: rank r draws the inputs of its own KV groups
+        w, first = shard_heads(w, rank, world)
+        seed_offset = first
+    else:
+        seed_offset = rank_seed_offset(rank)
+    layers = [Layer(w, dev, l, seed_offset=seed_offset) for l in range(w.layers)]
     torch.cuda.synchronize()
 
     # warm-up (also fixes the kept-block counts of this input)
@@ -292,12 +314,14 @@ def gpu_arm(args):
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if sharded else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 with planted salient keys)",
-        "config": {"workload": w.name, "batch": w.batch, "hq": w.hq, "hkv": w.hkv, "n": w.n,
+        "config": {"workload": w.name, "batch": w.batch, "hq": w_full.hq, "hkv": w_full.hkv,
+                   "n": w.n,
                    "d": w.d, "block": w.block, "segment": w.segment, "layers": w.layers,
                    "selection": f"{w.mode} {w.param}", "l2": "inputs larger than L2",
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"heads/{world}" if sharded else f"replicas x{world}"},
         "density": round(total_blocks / (len(layers) * w.batch * w.hq * w.nb * (w.nb + 1) / 2), 4),
         "breakdown_ms": {n: round(v, 4) for n, v in per.items()},
         "dense_attn_ms": round(dense_ms * len(layers), 4),

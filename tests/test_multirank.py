@@ -68,3 +68,59 @@ def test_single_process_throughput_needs_no_collective():
     import bench
     assert bench.job_throughput(2e12, 4.0) == (500.0, 4.0, 2e12)
     assert bench.rank_seed_offset(0) == 0 and bench.rank_seed_offset(3) == 3000
+
+
+def test_head_sharding_covers_every_kv_group_once():
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    from long_context_sparse_segment_b200.workloads import WORKLOADS
+    w = WORKLOADS["llama512k"]
+    for world in (1, 2, 4, 8):
+        heads = []
+        for rank in range(world):
+            ws, first = bench.shard_heads(w, rank, world)
+            assert ws.hq == ws.hkv * w.group and ws.n == w.n
+            heads += list(range(first, first + ws.hkv))
+        assert heads == list(range(w.hkv))
+    with pytest.raises(ValueError):
+        bench.shard_heads(w, 0, 3)
+
+
+def _sharded_worker(rank, world, port, out):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    from long_context_sparse_segment_b200.workloads import WORKLOADS
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w = WORKLOADS["llama128k"]
+        ws, _ = bench.shard_heads(w, rank, world)
+        # each rank's flops are its share of the sequence; strong scaling:
+        # the job's throughput is the whole sequence's flops over the slowest rank
+        flops = 1e12 * ws.hq / w.hq
+        value, ms, total = bench.job_throughput(flops, 5.0 + rank, dist, "cpu")
+        out.put((rank, value, ms, total))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_head_sharded_throughput_counts_the_sequence_once():
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [out.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, value, ms, total in results:
+        assert total == pytest.approx(1e12)      # the sequence's flops, once
+        assert ms == 6.0                         # the slower rank
+        assert value == pytest.approx(1e12 / 6e-3 / 1e12)
