@@ -16,12 +16,13 @@
 // works. TMEM (512 columns): S_A, S_B (P is written over the first 64
 // columns of its S as bf16 pairs), O_A, O_B. Q_A and Q_B stay in shared
 // memory. 384 threads, three warpgroups:
-//   warp 0, one thread   TMA: Q_A, Q_B, then K' and V' tiles in exactly the
+//   warp 0               TMA: Q_A, Q_B, then K' and V' tiles in exactly the
 //                        order the tensor core consumes them, into a K'
 //                        ring and a V' ring; a V' tile of an on-diagonal-
 //                        segment block brings the block's carried key
 //                        positions (512 bytes);
-//   warp 1, one thread   tcgen05.mma issue in the order above;
+//   warp 1               tcgen05.mma issue in the order above;
+//   (both warps run their loops warp-wide and issue from one elected lane)
 //   warps 4-7, 8-11      softmax of tile A, of tile B: one thread per query
 //                        row (TMEM lane), all 128 key columns of a block:
 //                        mask, row max, exp2 (MUFU), P to TMEM in two
