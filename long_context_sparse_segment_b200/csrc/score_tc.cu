@@ -29,8 +29,8 @@
 //                      halves and releases it once the second half is read,
 //                      so the tensor core refills it with the next tile
 //                      while the second half is worked on;
-//   warp 4W, lane 0    TMA: the probe rows once, then K tiles into a ring;
-//   warp 4W+1, lane 0  tcgen05.mma issue: per K tile and slice one
+//   warp 4W            TMA: the probe rows once, then K tiles into a ring;
+//   warp 4W+1          tcgen05.mma issue: per K tile and slice one
 //                      128 x 128 x d product, issued once the slice is free.
 // (Measured on B200: this beats releasing 64-column halves separately with
 // 128 x 64 products, and two warpgroups that each hold a whole slice.)
@@ -146,31 +146,39 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *s_tmem;
 
-  if (warp == pw && lane == 0) {
+  if (warp == pw) {
     // ------------------------------------------------------- TMA loads
+    // warp-wide loop, one elected lane issues the copies
+    const bool leader = elect_one();
     bool q_issued = false;
     int issued = 0;
     if (nt > 0) {
-      prefetch_map(&tmQ);
-      prefetch_map(&tmK);
-      // probe row r = gl * B + i is row n - B + i of query head h G + gl;
-      // 128-row tile r / 128 of the Q array, each tile stored as H boxes.
-      mbar_expect_tx(&bar->q_full, (uint32_t)W * C::TILE);
-      for (int gl = 0; gl < dm.G; ++gl) {
-        const int r0 = gl * dm.B;
-        const int grow = (b * dm.hq + h * dm.G + gl) * dm.n + dm.n - dm.B;
-        for (int hh = 0; hh < C::H; ++hh)
-          tma_load_2d(sQ + (size_t)(r0 / 128) * C::TILE + hh * C::HALF + (r0 % 128) * 128, &tmQ,
-                      &bar->q_full, hh * 64, grow);
+      if (leader) {
+        prefetch_map(&tmQ);
+        prefetch_map(&tmK);
+        // probe row r = gl * B + i is row n - B + i of query head h G + gl;
+        // 128-row tile r / 128 of the Q array, each tile stored as H boxes.
+        mbar_expect_tx(&bar->q_full, (uint32_t)W * C::TILE);
+        for (int gl = 0; gl < dm.G; ++gl) {
+          const int r0 = gl * dm.B;
+          const int grow = (b * dm.hq + h * dm.G + gl) * dm.n + dm.n - dm.B;
+          for (int hh = 0; hh < C::H; ++hh)
+            tma_load_2d(sQ + (size_t)(r0 / 128) * C::TILE + hh * C::HALF + (r0 % 128) * 128,
+                        &tmQ, &bar->q_full, hh * 64, grow);
+        }
       }
+      __syncwarp();
       q_issued = true;
       for (int it = 0; it < nt; ++it) {
         const int s = it % C::KS, u = it / C::KS;
-        if (u > 0 && !mbar_wait(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 51)) break;
-        mbar_expect_tx(&bar->k_full[s], C::TILE);
-        for (int hh = 0; hh < C::H; ++hh)
-          tma_load_2d(sK + (size_t)s * C::TILE + hh * C::HALF, &tmK, &bar->k_full[s], hh * 64,
-                      bh * dm.n + (t0 + it) * kKT);
+        if (u > 0 && !mbar_wait_warp(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 51)) break;
+        if (leader) {
+          mbar_expect_tx(&bar->k_full[s], C::TILE);
+          for (int hh = 0; hh < C::H; ++hh)
+            tma_load_2d(sK + (size_t)s * C::TILE + hh * C::HALF, &tmK, &bar->k_full[s], hh * 64,
+                        bh * dm.n + (t0 + it) * kKT);
+        }
+        __syncwarp();
         issued = it + 1;
       }
     }
@@ -179,23 +187,26 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     if (q_issued) mbar_wait(&bar->q_full, 0, &never, nullptr);
     for (int t = issued > C::KS ? issued - C::KS : 0; t < issued; ++t)
       mbar_wait(&bar->k_full[t % C::KS], (t / C::KS) & 1, &never, nullptr);
-  } else if (warp == pw + 1 && lane == 0) {
+  } else if (warp == pw + 1) {
     // -------------------------------------------------------- MMA issue
+    // warp-wide loop (uniform waits and descriptor arithmetic), one elected
+    // lane issues every MMA and commit.
     // Both operands K-major with the 128-byte swizzle; a k-step of 16 moves
     // 32 bytes inside a 64-column box, every 4 steps to the next box.
+    const bool leader = elect_one();
     constexpr uint32_t kId = idesc_bf16(128, kKT, false);
     const uint32_t hi = sw128_desc_hi(1024);
     const uint32_t lo_q = sw128_desc_lo(smem_u32(sQ), 16);
     const uint32_t lo_k = sw128_desc_lo(smem_u32(sK), 16);
-    if (nt > 0 && mbar_wait(&bar->q_full, 0, s_abort, err, 52)) {
+    if (nt > 0 && mbar_wait_warp(&bar->q_full, 0, s_abort, err, 52)) {
       tc_fence_after();
       int ks = 0, kph = 0;
       bool ok = true;
       for (int it = 0; it < nt && ok; ++it) {
-        if (!mbar_wait(&bar->k_full[ks], kph, s_abort, err, 53)) break;
+        if (!mbar_wait_warp(&bar->k_full[ks], kph, s_abort, err, 53)) break;
         tc_fence_after();
         for (int w = 0; w < W; ++w) {
-          if (it > 0 && !mbar_wait(&bar->s_free[w], (it - 1) & 1, s_abort, err, 54)) {
+          if (it > 0 && !mbar_wait_warp(&bar->s_free[w], (it - 1) & 1, s_abort, err, 54)) {
             ok = false;
             break;
           }
@@ -204,21 +215,26 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           // pass 2: A = the K tile, B = Q rows of slice w (keys x rows)
           const uint32_t lq = lo_q + w * (C::TILE >> 4), lk = lo_k + ks * (C::TILE >> 4);
           const uint32_t la = PASS == 0 ? lq : lk, lb = PASS == 0 ? lk : lq;
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t step = ((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4;
-            mma_ss(tbase + w * 128, desc_words(la + step, hi), desc_words(lb + step, hi), kId,
-                   kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t step = ((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4;
+              mma_ss(tbase + w * 128, desc_words(la + step, hi), desc_words(lb + step, hi), kId,
+                     kk > 0);
+            }
+            mma_commit(&bar->s_full[w]);
           }
-          mma_commit(&bar->s_full[w]);
+          __syncwarp();
         }
         if (!ok) break;
-        mma_commit(&bar->k_empty[ks]);
+        if (leader) mma_commit(&bar->k_empty[ks]);
+        __syncwarp();
         if (++ks == C::KS) ks = 0, kph ^= 1;
       }
     }
     // drain: every MMA issued here completes before TMEM is released
-    mma_commit(&bar->mma_done);
+    if (leader) mma_commit(&bar->mma_done);
+    __syncwarp();
     int never = 0;
     mbar_wait(&bar->mma_done, 0, &never, nullptr);
   } else if (warp < pw) {
