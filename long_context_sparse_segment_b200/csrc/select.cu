@@ -11,7 +11,8 @@
 // rows). Two kernels:
 //   scores: a_IJ = sigma * qbar_I . kbar_J for every admissible (I, J) on the
 //     fp64 tensor cores (mma.sync m8n8k4, 64 x 64 tiles of query blocks by
-//     key blocks, d staged once in shared memory), written to the workspace
+//     key blocks, d staged 64 columns at a time in shared memory so three tiles
+//     run per SM), written to the workspace
 //     as 64-bit order keys: every pooled key block is read once per tile
 //     instead of once per query block;
 //   selection: one warp per query block decides, without sorting, reading
@@ -106,11 +107,12 @@ __device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
 // 8 warps as 2 x 4: a warp owns 32 query blocks x 16 key blocks, i.e. 4 x 2
 // m8n8k4 products per 4-wide step of d.
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads)
     scores_kernel(const double *__restrict__ qsum, const double *__restrict__ ksum, Dims dm,
                   double sigma, unsigned long long *__restrict__ keys) {
   extern __shared__ __align__(16) unsigned char smem[];
-  constexpr int LD = D + kPad;
+  constexpr int KC = 64;           // columns of d staged at a time (three CTAs per SM)
+  constexpr int LD = KC + kPad;
   double *As = reinterpret_cast<double *>(smem);  // [kTile][LD] query block means
   double *Bs = As + kTile * LD;                   // [kTile][LD] key block means
   const int nb = dm.nb;
@@ -121,12 +123,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (C0 >= min(nb, (last / dm.spb + 1) * dm.spb)) return;  // nothing admissible here
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const double inv_b = 1.0 / (double)dm.B;  // a power of two: exact
-  for (int e = tid; e < kTile * D; e += kThreads) {
-    const int r = e / D, c = e % D;
-    As[r * LD + c] = R0 + r < nb ? qsum[((size_t)bg * nb + R0 + r) * D + c] * inv_b : 0.0;
-    Bs[r * LD + c] = C0 + r < nb ? ksum[((size_t)kv * nb + C0 + r) * D + c] * inv_b : 0.0;
-  }
-  __syncthreads();
   const int wr = (w >> 2) * 32, wc = (w & 3) * 16;
   double acc[4][2][2];
 #pragma unroll
@@ -135,17 +131,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int nt = 0; nt < 2; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = 0.0;
   const double *ap = As + (wr + (lane >> 2)) * LD + (lane & 3);
   const double *bp = Bs + (wc + (lane >> 2)) * LD + (lane & 3);
+#pragma unroll 1
+  for (int k0 = 0; k0 < D; k0 += KC) {
+    if (k0) __syncthreads();  // the previous columns are consumed
+    for (int e = tid; e < kTile * KC; e += kThreads) {
+      const int r = e / KC, c = e % KC;
+      As[r * LD + c] = R0 + r < nb ? qsum[((size_t)bg * nb + R0 + r) * D + k0 + c] * inv_b : 0.0;
+      Bs[r * LD + c] = C0 + r < nb ? ksum[((size_t)kv * nb + C0 + r) * D + k0 + c] * inv_b : 0.0;
+    }
+    __syncthreads();
 #pragma unroll 4
-  for (int k = 0; k < D; k += 4) {
-    double af[4], bf[2];
+    for (int k = 0; k < KC; k += 4) {
+      double af[4], bf[2];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt) af[mt] = ap[mt * 8 * LD + k];
+      for (int mt = 0; mt < 4; ++mt) af[mt] = ap[mt * 8 * LD + k];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) bf[nt] = bp[nt * 8 * LD + k];
+      for (int nt = 0; nt < 2; ++nt) bf[nt] = bp[nt * 8 * LD + k];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
+      for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) dmma_8x8x4(acc[mt][nt], af[mt], bf[nt]);
+        for (int nt = 0; nt < 2; ++nt) dmma_8x8x4(acc[mt][nt], af[mt], bf[nt]);
+    }
   }
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
@@ -374,7 +380,7 @@ cudaError_t launch_select(const Dims &dm, const double *qsum, const double *ksum
   cudaError_t e;
   if (scored) {
     auto sk = dm.d == 64 ? scores_kernel<64> : scores_kernel<128>;
-    const size_t ssm = (size_t)2 * kTile * (dm.d + kPad) * 8;
+    const size_t ssm = (size_t)2 * kTile * (64 + kPad) * 8;
     e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
     if (e != cudaSuccess) return e;
     const int tiles = (dm.nb + kTile - 1) / kTile;
