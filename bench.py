@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N > 1: every rank runs the whole workload (weak scaling), or "
                          "the KV groups of one workload are split over the ranks (strong)")
+    ap.add_argument("--gather-kv", action="store_true",
+                    help="the forward reads K, V through the key order (pbs_attn_fwd_gather); "
+                         "the permutation writes only the order and block sums")
     ap.add_argument("--profile", action="store_true",
                     help="time the steps only (no dense, end-to-end or CPU legs), for ncu")
     return ap.parse_args()
@@ -159,8 +162,9 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- GPU arm
 class Layer:
-    def __init__(self, w, dev, layer, seed_offset):
+    def __init__(self, w, dev, layer, seed_offset, gather_kv=False):
         self.w = w
+        self.gather_kv = gather_kv  # the forward reads K, V through the key order
         self.q, self.k, self.v, _ = make_inputs(w, dev, layer=layer, seed=w.seed + layer + seed_offset)
         self.out = None
 
@@ -179,15 +183,19 @@ def run_layer(layer, ev=None):
     imp = pbs.score(layer.q, layer.k, B, S)
     mark("score", 1)
     mark("permute", 0)
-    perm = pbs.permute(imp, layer.k, layer.v, B, S, hq=w.hq)
+    perm = pbs.permute(imp, layer.k, layer.v, B, S, hq=w.hq, materialize=not layer.gather_kv)
     mark("permute", 1)
     mark("select", 0)
     idx, cnt, _ = pbs.select_blocks(layer.q, perm["k_perm"], perm["kbar_sum"], B, S, w.mode,
                                     w.param)
     mark("select", 1)
     mark("attn", 0)
-    o = pbs.attn_fwd(layer.q, perm["k_perm"], perm["v_perm"], perm["kpos"], None, idx, cnt, B,
-                     S, out=layer.out)
+    if layer.gather_kv:
+        o = pbs.attn_fwd_gather(layer.q, layer.k, layer.v, perm["kpos"], None, idx, cnt, B, S,
+                                out=layer.out)
+    else:
+        o = pbs.attn_fwd(layer.q, perm["k_perm"], perm["v_perm"], perm["kpos"], None, idx, cnt,
+                         B, S, out=layer.out)
     mark("attn", 1)
     layer.out = o
     return o, cnt
@@ -266,7 +274,8 @@ def gpu_arm(args):
         seed_offset = first
     else:
         seed_offset = rank_seed_offset(rank)
-    layers = [Layer(w, dev, l, seed_offset=seed_offset) for l in range(w.layers)]
+    layers = [Layer(w, dev, l, seed_offset=seed_offset, gather_kv=args.gather_kv)
+              for l in range(w.layers)]
     torch.cuda.synchronize()
 
     # warm-up (also fixes the kept-block counts of this input)
@@ -321,7 +330,8 @@ def gpu_arm(args):
                    "n": w.n,
                    "d": w.d, "block": w.block, "segment": w.segment, "layers": w.layers,
                    "selection": f"{w.mode} {w.param}", "l2": "inputs larger than L2",
-                   "parallelism": f"heads/{world}" if sharded else f"replicas x{world}"},
+                   "parallelism": f"heads/{world}" if sharded else f"replicas x{world}",
+                   "kv": "gathered inside the forward" if args.gather_kv else "permuted copies"},
         "density": round(total_blocks / (len(layers) * w.batch * w.hq * w.nb * (w.nb + 1) / 2), 4),
         "breakdown_ms": {n: round(v, 4) for n, v in per.items()},
         "dense_attn_ms": round(dense_ms * len(layers), 4),
@@ -334,7 +344,8 @@ def gpu_arm(args):
         "roofline": {"kernel": "pbs_attn_fwd", "bound": "tensor",
                      "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peak, 4), "peak_kind":
-                     f"{pk_kind} bf16 dense, sustained", "traffic": traffic_for(w)},
+                     f"{pk_kind} bf16 dense, sustained",
+                     "traffic": None if args.gather_kv else traffic_for(w)},
     }
     if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.profile):
         line["cpu_baseline"] = cpu_baseline(w, layers[0], total_blocks / len(layers))

@@ -11,6 +11,7 @@
  *   pbs_attn_fwd       causal block-sparse attention on the permuted keys
  *   pbs_unpermute      inverse permutation of the output rows
  *   pbs_attn_fwd_unpermute  the last two fused: rows written in place
+ *   pbs_attn_fwd_gather     the forward reading K, V through kpos (no K', V')
  *   pbs_attention_host the whole path on host buffers, copies overlapped
  *   pbs_block_mass, pbs_coverage  diagnostics: attention coverage and
  *                      block-level density
@@ -148,7 +149,9 @@ pbs_status pbs_score_static(const void *q, const void *k, float *imp, pbs_shape 
  *   imp         [batch, hkv, n] fp32 (no NaN)
  *   k, v        [batch, hkv, n, d] bf16
  *   q, q_perm   [batch, hq, n, d] bf16, both NULL or both non-NULL
- *   k_perm, v_perm  [batch, hkv, n, d] bf16, written
+ *   k_perm, v_perm  [batch, hkv, n, d] bf16, written; both NULL: only kpos
+ *               and kbar_sum are produced (for pbs_attn_fwd_gather, which
+ *               reads K and V through kpos); one NULL is PBS_ERR_INVALID_ARG
  *   kpos        [batch, hkv, n] int32, written
  *   kbar_sum    [batch, hkv, n/B, d] fp64, written if non-NULL
  */
@@ -243,6 +246,33 @@ pbs_status pbs_attn_fwd_unpermute(const void *q_perm, const void *k_perm,
                                   const int32_t *qpos, const int32_t *blk_idx,
                                   const int32_t *blk_cnt, void *out, float *lse,
                                   pbs_shape s, float scale, pbs_stream_t st);
+
+/*
+ * pbs_attn_fwd_gather - pbs_attn_fwd on the natural K and V, each permuted
+ * key read from its original row: key slot p of KV head (b, h) is row
+ * kpos[b, h, p] of k and v. The result is bit-identical to pbs_attn_fwd
+ * given k_perm = k[kpos], v_perm = v[kpos], without writing or re-reading
+ * those copies. Source: as for pbs_attn_fwd; a segment-local permutation
+ * (gist.science summary, "Methodik" 2) only decides which rows form each
+ * key block, so the forward may fetch them by index. Fetching on the fly is
+ * this library's choice (the pages gather before the forward).
+ *
+ *   q_or_qperm  [batch, hq, n, d] bf16: Q, or Q' in permuted-query mode
+ *   k, v        [batch, hkv, n, d] bf16, natural order
+ *   kpos        [batch, hkv, n] int32, required: every segment holds a
+ *               permutation of its own positions (as from pbs_permute); a
+ *               position outside its block's segment is reported as
+ *               PBS_ERR_DEVICE_ASSERT and the key's own row is read instead
+ *   qpos, blk_idx, blk_cnt, out, lse  as for pbs_attn_fwd
+ *   unpermute   nonzero: rows written at qpos as by pbs_attn_fwd_unpermute
+ *               (then `out` must not be q_or_qperm, k or v)
+ */
+pbs_status pbs_attn_fwd_gather(const void *q_or_qperm, const void *k,
+                               const void *v, const int32_t *kpos,
+                               const int32_t *qpos, const int32_t *blk_idx,
+                               const int32_t *blk_cnt, void *out, float *lse,
+                               pbs_shape s, float scale, int unpermute,
+                               pbs_stream_t st);
 
 /*
  * pbs_unpermute - inverse permutation of the output rows.

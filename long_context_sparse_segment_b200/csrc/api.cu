@@ -161,11 +161,14 @@ pbs_status pbs_permute(const float *imp, const void *k, const void *v, const voi
   pbs_status r = check_shape(s, &dm);
   if (r != PBS_OK) return r;
   if (empty(dm)) return PBS_OK;
-  if (!imp || !k || !v || !k_perm || !v_perm || !kpos) return PBS_ERR_INVALID_ARG;
+  if (!imp || !k || !v || !kpos) return PBS_ERR_INVALID_ARG;
+  // K' and V' are both written or (order only: the forward gathers) neither
+  if ((k_perm == nullptr) != (v_perm == nullptr)) return PBS_ERR_INVALID_ARG;
   if ((q == nullptr) != (q_perm == nullptr)) return PBS_ERR_INVALID_ARG;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(k_perm) || !aligned16(v_perm) ||
-      !aligned16(kpos) || (q && (!aligned16(q) || !aligned16(q_perm))) ||
-      (kbar_sum && !aligned16(kbar_sum)) || ((uintptr_t)imp & 3u))
+  if (!aligned16(k) || !aligned16(v) || (k_perm && !aligned16(k_perm)) ||
+      (v_perm && !aligned16(v_perm)) || !aligned16(kpos) ||
+      (q && (!aligned16(q) || !aligned16(q_perm))) || (kbar_sum && !aligned16(kbar_sum)) ||
+      ((uintptr_t)imp & 3u))
     return PBS_ERR_INVALID_ARG;
   if (k == k_perm || v == v_perm || (q && q == q_perm)) return PBS_ERR_INVALID_ARG;
   int *err = error_word();
@@ -223,12 +226,12 @@ namespace {
 pbs_status attn_fwd(const void *q_or_qperm, const void *k_perm, const void *v_perm,
                     const int32_t *kpos, const int32_t *qpos, const int32_t *blk_idx,
                     const int32_t *blk_cnt, void *out, float *lse, pbs_shape s, float scale,
-                    bool scatter, pbs_stream_t st) {
+                    bool scatter, bool gather, pbs_stream_t st) {
   Dims dm;
   pbs_status r = check_shape(s, &dm);
   if (r != PBS_OK) return r;
   if (empty(dm)) return PBS_OK;
-  if (!q_or_qperm || !k_perm || !v_perm || !blk_idx || !blk_cnt || !out)
+  if (!q_or_qperm || !k_perm || !v_perm || !blk_idx || !blk_cnt || !out || (gather && !kpos))
     return PBS_ERR_INVALID_ARG;
   if (!aligned16(q_or_qperm) || !aligned16(k_perm) || !aligned16(v_perm) || !aligned16(out) ||
       (kpos && !aligned16(kpos)) || (qpos && ((uintptr_t)qpos & 3u)) ||
@@ -239,7 +242,7 @@ pbs_status attn_fwd(const void *q_or_qperm, const void *k_perm, const void *v_pe
   int *err = error_word();
   const float sigma = (float)resolve_sigma(scale, dm.d);
   return cuda_status(launch_attn(dm, q_or_qperm, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt,
-                                 out, lse, sigma, err, scatter && qpos, (cudaStream_t)st));
+                                 out, lse, sigma, err, scatter && qpos, gather, (cudaStream_t)st));
 }
 
 }  // namespace
@@ -249,7 +252,7 @@ pbs_status pbs_attn_fwd(const void *q_or_qperm, const void *k_perm, const void *
                         const int32_t *blk_cnt, void *out, float *lse, pbs_shape s, float scale,
                         pbs_stream_t st) {
   return attn_fwd(q_or_qperm, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt, out, lse, s, scale,
-                  false, st);
+                  false, false, st);
 }
 
 pbs_status pbs_attn_fwd_unpermute(const void *q_perm, const void *k_perm, const void *v_perm,
@@ -257,7 +260,15 @@ pbs_status pbs_attn_fwd_unpermute(const void *q_perm, const void *k_perm, const 
                                   const int32_t *blk_idx, const int32_t *blk_cnt, void *out,
                                   float *lse, pbs_shape s, float scale, pbs_stream_t st) {
   return attn_fwd(q_perm, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt, out, lse, s, scale, true,
-                  st);
+                  false, st);
+}
+
+pbs_status pbs_attn_fwd_gather(const void *q_or_qperm, const void *k, const void *v,
+                               const int32_t *kpos, const int32_t *qpos, const int32_t *blk_idx,
+                               const int32_t *blk_cnt, void *out, float *lse, pbs_shape s,
+                               float scale, int unpermute, pbs_stream_t st) {
+  return attn_fwd(q_or_qperm, k, v, kpos, qpos, blk_idx, blk_cnt, out, lse, s, scale,
+                  unpermute != 0, true, st);
 }
 
 pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out, pbs_shape s,
@@ -338,7 +349,7 @@ pbs_status pbs_attention_host(const void *q, const void *k, const void *v, void 
                         (uint8_t *)sl.qsum + select_qsum_bytes(g), err, cs);
     if (e == cudaSuccess)
       e = launch_attn(g, sl.q, sl.kp, sl.vp, sl.kpos, nullptr, sl.idx, sl.cnt, sl.o, nullptr,
-                      sigma_f, err, false, cs);
+                      sigma_f, err, false, false, cs);
     if (e == cudaSuccess) e = cudaEventRecord(ev[1][sid], cs);
     // out
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ds, ev[1][sid], 0);

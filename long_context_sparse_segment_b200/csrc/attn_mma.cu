@@ -44,13 +44,35 @@ __device__ __forceinline__ void load_tile(bf16 *dst, const bf16 *src, int tid) {
   }
 }
 
+// The same tile with row r read from row pos[r] of `base` (the carried key
+// positions of block J: the permutation applied on the fly). A position
+// outside the block's segment [seg0, seg0 + span) is reported and replaced by
+// the key's own index p0 + r.
+template <int D, int BB>
+__device__ __forceinline__ void load_tile_rows(bf16 *dst, const bf16 *base,
+                                               const int32_t *__restrict__ pos, int p0, int seg0,
+                                               int span, int tid, int *err) {
+  constexpr int RC = D / 8;
+  for (int i = tid; i < BB * RC; i += MmaCfg<D, BB>::kThreads) {
+    const int r = i / RC, c = i % RC;
+    int src = __ldg(pos + r);
+    if ((unsigned)(src - seg0) >= (unsigned)span) {
+      report(err, PBS_ERR_DEVICE_ASSERT);
+      src = p0 + r;
+    }
+    cp_async16(&dst[swz<D>(r, c * 8)], base + (size_t)src * D + c * 8);
+  }
+}
+
+// gather != 0: kp and vp are the natural K and V, read through kpos.
 template <int D, int BB>
 __global__ void __launch_bounds__(MmaCfg<D, BB>::kThreads, 1)
     attn_mma_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ kp,
                     const bf16 *__restrict__ vp, const int32_t *__restrict__ kpos,
                     const int32_t *__restrict__ qpos, const int32_t *__restrict__ blk_idx,
                     const int32_t *__restrict__ blk_cnt, bf16 *__restrict__ out,
-                    float *__restrict__ lse, Dims dm, float sl2, int *err, int scatter) {
+                    float *__restrict__ lse, Dims dm, float sl2, int *err, int scatter,
+                    int gather) {
   using C = MmaCfg<D, BB>;
   extern __shared__ __align__(128) uint8_t smem[];
   bf16 *Qs = reinterpret_cast<bf16 *>(smem);
@@ -83,8 +105,18 @@ __global__ void __launch_bounds__(MmaCfg<D, BB>::kThreads, 1)
       report(err, PBS_ERR_DEVICE_ASSERT);
       J = 0;
     }
-    load_tile<D, BB>(Ks + stage * C::kTile, kp + (krow0 + (size_t)J * BB) * D, tid);
-    load_tile<D, BB>(Vs + stage * C::kTile, vp + (krow0 + (size_t)J * BB) * D, tid);
+    if (gather) {
+      const int32_t *pos = kpos + krow0 + (size_t)J * BB;
+      const int seg0 = (J / dm.spb) * dm.S;
+      const int span = min(dm.S, dm.n - seg0);  // the last segment may be short
+      load_tile_rows<D, BB>(Ks + stage * C::kTile, kp + krow0 * D, pos, J * BB, seg0, span, tid,
+                            err);
+      load_tile_rows<D, BB>(Vs + stage * C::kTile, vp + krow0 * D, pos, J * BB, seg0, span, tid,
+                            err);
+    } else {
+      load_tile<D, BB>(Ks + stage * C::kTile, kp + (krow0 + (size_t)J * BB) * D, tid);
+      load_tile<D, BB>(Vs + stage * C::kTile, vp + (krow0 + (size_t)J * BB) * D, tid);
+    }
     for (int i = tid; i < BB / 4; i += C::kThreads) {
       if (kpos)
         cp_async16(&Ps[stage * BB + i * 4], kpos + krow0 + (size_t)J * BB + i * 4);
@@ -234,15 +266,17 @@ __global__ void __launch_bounds__(MmaCfg<D, BB>::kThreads, 1)
 template <int D, int BB>
 cudaError_t run(const Dims &dm, const void *q, const void *kp, const void *vp,
                 const int32_t *kpos, const int32_t *qpos, const int32_t *idx, const int32_t *cnt,
-                void *out, float *lse, float sigma, int *err, bool scatter, cudaStream_t st) {
+                void *out, float *lse, float sigma, int *err, bool scatter, bool gather,
+                cudaStream_t st) {
   using C = MmaCfg<D, BB>;
+  if (gather && !kpos) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<D, BB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)dm.b * dm.hq * dm.nb;
   attn_mma_kernel<D, BB><<<grid, C::kThreads, C::smem, st>>>(
       (const bf16 *)q, (const bf16 *)kp, (const bf16 *)vp, kpos, qpos, idx, cnt, (bf16 *)out,
-      lse, dm, sigma * kLog2e, err, scatter ? 1 : 0);
+      lse, dm, sigma * kLog2e, err, scatter ? 1 : 0, gather ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -251,14 +285,18 @@ cudaError_t run(const Dims &dm, const void *q, const void *kp, const void *vp,
 cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                             const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            bool scatter, cudaStream_t st) {
+                            bool scatter, bool gather, cudaStream_t st) {
   if (dm.d == 64 && dm.B == 64)
-    return run<64, 64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter, st);
+    return run<64, 64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter,
+                       gather, st);
   if (dm.d == 64 && dm.B == 128)
-    return run<64, 128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter, st);
+    return run<64, 128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter,
+                        gather, st);
   if (dm.d == 128 && dm.B == 64)
-    return run<128, 64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter, st);
-  return run<128, 128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter, st);
+    return run<128, 64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter,
+                        gather, st);
+  return run<128, 128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter,
+                       gather, st);
 }
 
 }  // namespace pbs
@@ -274,28 +312,31 @@ namespace pbs {
 // one-tile kernel then runs instead.
 // PBS_FAULT_INJECT=timeout makes the tcgen05 kernels skip their first K'
 // load, so that their bounded waits run out and they report
-// PBS_ERR_TIMEOUT (used by the failure-detection test).
+// PBS_ERR_TIMEOUT (used by the failure-detection test). With `gather` (keys
+// read through kpos) the one-tile kernel is not used: the warp-MMA kernel
+// serves what the two-tile kernel does not.
 cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const void *vp,
                         const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                         const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                        bool scatter, cudaStream_t st) {
+                        bool scatter, bool gather, cudaStream_t st) {
   const char *fwd = getenv("PBS_FORWARD");
   const bool force_mma = fwd && strcmp(fwd, "mma") == 0;
   const bool force_tc1 = fwd && strcmp(fwd, "tc1") == 0;
   if (attn_tc_supported(dm) && !force_mma) {
     const char *fi = getenv("PBS_FAULT_INJECT");
     const int fault = (fi && strcmp(fi, "timeout") == 0) ? 1 : 0;
-    if (!force_tc1) {
+    if (!force_tc1 || gather) {
       const cudaError_t e =
           launch_attn_tc2(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
-                          scatter, st);
+                          scatter, gather, st);
       if (e != cudaErrorInvalidConfiguration) return e;
     }
-    return launch_attn_tc(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
-                          scatter, st);
+    if (!gather)
+      return launch_attn_tc(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+                            scatter, st);
   }
   return launch_attn_mma(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, scatter,
-                         st);
+                         gather, st);
 }
 
 }  // namespace pbs

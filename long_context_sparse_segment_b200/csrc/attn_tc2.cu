@@ -23,6 +23,11 @@
 //                        positions (512 bytes);
 //   warp 1               tcgen05.mma issue in the order above;
 //   (both warps run their loops warp-wide and issue from one elected lane)
+//   warps 2, 3           idle, or with GATHER (pbs_attn_fwd_gather) the K
+//                        and V tiles: each row read from the natural K, V at
+//                        its carried position with cp.async, into the
+//                        layout the TMA would write (warp 0 then loads Q
+//                        only).
 //   warps 4-7, 8-11      softmax of tile A, of tile B: one thread per query
 //                        row (TMEM lane), all 128 key columns of a block:
 //                        mask, row max, exp2 (MUFU), P to TMEM in two
@@ -135,7 +140,28 @@ __device__ __forceinline__ int stream_pos(int x, int j, int cA, int cB) {
   return x == 0 ? j + min(j, cB) : j + min(j + 1, cA);
 }
 
-template <int D>
+// Carried positions of keys 64 w + lane and 64 w + 32 + lane of block J of
+// KV head bh (w = 0, 1: the two gathering warps). A position outside block
+// J's segment is reported and replaced by the key's own index.
+__device__ __forceinline__ int2 carried_rows(const int32_t *__restrict__ kpos, int bh, int J,
+                                             int w, int lane, const Dims &dm, int *err) {
+  const int p0 = J * kBN + 64 * w + lane;
+  const int32_t *p = kpos + (size_t)bh * dm.n + p0;
+  int2 r = make_int2(__ldg(p), __ldg(p + 32));
+  const int seg0 = (J / dm.spb) * dm.S;
+  const unsigned span = (unsigned)min(dm.S, dm.n - seg0);  // the last segment may be short
+  if ((unsigned)(r.x - seg0) >= span || (unsigned)(r.y - seg0) >= span) {
+    report(err, PBS_ERR_DEVICE_ASSERT);
+    r = make_int2(p0, p0 + 32);
+  }
+  return r;
+}
+
+// GATHER: the permutation is applied on the fly. kg and vg are the natural
+// K and V; warps 2 and 3 fetch each block's rows by their carried positions
+// with cp.async into the same swizzled tiles the TMA would write (no K', V'
+// copies); tmK and tmV are unused.
+template <int D, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc2_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK,
@@ -143,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int32_t *__restrict__ qpos, const int32_t *__restrict__ blk_idx,
                     const int32_t *__restrict__ blk_cnt, bf16 *__restrict__ out,
                     float *__restrict__ lse, Dims dm, float sl2, int *err, int fault,
-                    int scatter) {
+                    int scatter, const bf16 *__restrict__ kg, const bf16 *__restrict__ vg) {
   using C = Cfg2<D>;
   constexpr int KS = C::KS, VS = C::VS;
   extern __shared__ uint8_t smem_raw[];
@@ -166,12 +192,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&bar->q_full, 1);
+    // full: the TMA's expect-tx arrival, or one cp.async arrival per
+    // gathering thread
+    const int fill_count = GATHER ? 64 : 1;
     for (int s = 0; s < KS; ++s) {
-      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->k_full[s], fill_count);
       mbar_init(&bar->k_empty[s], 1);
     }
     for (int s = 0; s < VS; ++s) {
-      mbar_init(&bar->v_full[s], 1);
+      mbar_init(&bar->v_full[s], fill_count);
       mbar_init(&bar->v_empty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -206,8 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kseq = 0, vseq = 0;
     if (cmax > 0) {
       prefetch_map(&tmQ);
-      prefetch_map(&tmK);
-      prefetch_map(&tmV);
+      if (!GATHER) {
+        prefetch_map(&tmK);
+        prefetch_map(&tmV);
+      }
       if (leader) {
         mbar_expect_tx(&bar->q_full, ((cA > 0) + (cB > 0)) * C::TILE);
         for (int x = 0; x < 2; ++x) {
@@ -255,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++vseq;
         return true;
       };
-      bool ok = true;
-      if (cA > 0) ok = load_k(tA, 0);
+      bool ok = !GATHER;  // with GATHER, warps 2 and 3 load K and V
+      if (ok && cA > 0) ok = load_k(tA, 0);
       if (ok && cB > 0) ok = load_k(tB, 0);
       for (int j = 0; j < cmax && ok; ++j)
         for (int x = 0; x < 2 && ok; ++x) {
@@ -291,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto qk = [&](int x) -> bool {
       if (!mbar_wait_warp(&bar->k_full[ks], kph, s_abort, err, 32)) return false;
       tc_fence_after();
+      if constexpr (GATHER) fence_proxy_async_smem();  // rows written by cp.async
       const uint32_t lq = lo_q + x * (C::TILE >> 4), lk = lo_k + ks * (C::TILE >> 4);
       if (leader) {
 #pragma unroll
@@ -314,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_warp(&bar->p_full[x][0], j & 1, s_abort, err, 33)) return false;
       if (!mbar_wait_warp(&bar->v_full[vs], vph, s_abort, err, 34)) return false;
       tc_fence_after();
+      if constexpr (GATHER) fence_proxy_async_smem();
       const uint32_t lv = lo_v + vs * (C::TILE >> 4);
       for (int h = 0; h < 2; ++h) {
         if (h == 1) {
@@ -355,6 +388,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     int never = 0;
     mbar_wait(&bar->mma_done, 0, &never, nullptr);
+  } else if (GATHER) {
+    // ------------------------------------------- K, V gathers (warps 2, 3)
+    // The K and V tiles in the TMA producer's order, each row read from its
+    // carried position: warp 2 fills rows 0-63 of every tile, warp 3 rows
+    // 64-127. A warp instruction moves 32 16-byte chunks (whole rows, 2 of
+    // them at d = 128) into the 128-byte-swizzled layout; each thread's
+    // cp.async arrival on the tile's full barrier (64 expected) lands when
+    // its copies have. The positions of a K block are kept for the V block
+    // of the same tile that follows it.
+    const int gw = warp - 2;
+    constexpr int CPR = D / 8;    // 16-byte chunks per row
+    constexpr int RPI = 32 / CPR; // rows per warp instruction
+    const int sub = lane / CPR, ch = lane % CPR;
+    const uint32_t col = (uint32_t)(ch >> 3) * C::HALF;  // 128-byte column block
+    const int cc = ch & 7;
+    int2 rows_a = make_int2(0, 0), rows_b = rows_a;
+    int kseq = 0, vseq = 0;
+    auto fill = [&](uint8_t *tile, const bf16 *src, int bh, int2 r) {
+      const bf16 *head = src + (size_t)bh * dm.n * D + ch * 8;
+#pragma unroll 4
+      for (int it = 0; it < 64 / RPI; ++it) {
+        const int rl = it * RPI + sub;  // 0-63, warp-uniform half of r
+        const int pos = __shfl_sync(0xffffffffu, it * RPI < 32 ? r.x : r.y, rl & 31);
+        const int row = 64 * gw + rl;
+        cp_async16(tile + col + row * 128 + ((cc ^ (row & 7)) << 4), head + (size_t)pos * D);
+      }
+    };
+    auto load_k = [&](const Tile &t, int x, int j) -> bool {
+      const int s = kseq % KS, u = kseq / KS;
+      const int J = checked_block(t, j, dm, gw == 0 && lane == 0 ? err : nullptr);
+      // the positions are read before the wait for the slot: their latency
+      // hides behind it
+      const int2 r = carried_rows(kpos, t.bh, J, gw, lane, dm, err);
+      if (x) rows_b = r;
+      else rows_a = r;
+      if (u > 0 && !mbar_wait_warp(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 12))
+        return false;
+      if (!(fault == 1 && kseq == 0)) {
+        fill(sK + s * C::TILE, kg, t.bh, r);
+        cp_async_mbar_arrive(&bar->k_full[s]);
+      }
+      ++kseq;
+      return true;
+    };
+    auto load_v = [&](const Tile &t, int x, int j) -> bool {
+      const int s = vseq % VS, u = vseq / VS;
+      if (u > 0 && !mbar_wait_warp(&bar->v_empty[s], (u - 1) & 1, s_abort, err, 22))
+        return false;
+      const int J = checked_block(t, j, dm, nullptr);
+      fill(sV + s * C::TILE, vg, t.bh, x ? rows_b : rows_a);
+      if (J / dm.spb == t.segI && lane < 16)  // the mask's positions, 4 per lane
+        cp_async16(sKP + s * kBN + 64 * gw + 4 * lane,
+                   kpos + (size_t)t.bh * dm.n + (size_t)J * kBN + 64 * gw + 4 * lane);
+      cp_async_mbar_arrive(&bar->v_full[s]);
+      ++vseq;
+      return true;
+    };
+    bool ok = true;
+    if (cA > 0) ok = load_k(tA, 0, 0);
+    if (ok && cB > 0) ok = load_k(tB, 1, 0);
+    for (int j = 0; j < cmax && ok; ++j)
+      for (int x = 0; x < 2 && ok; ++x) {
+        const Tile &t = x ? tB : tA;
+        if (j >= t.count) continue;
+        ok = load_v(t, x, j);
+        if (ok && j + 1 < t.count) ok = load_k(t, x, j + 1);
+      }
+    cp_async_wait_all();  // every copy lands before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -522,31 +623,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool GATHER>
 cudaError_t run2(const Dims &dm, const void *q, const void *kp, const void *vp,
                  const int32_t *kpos, const int32_t *qpos, const int32_t *idx, const int32_t *cnt,
                  void *out, float *lse, float sigma, int *err, int fault, bool scatter,
                  cudaStream_t st) {
+  if (GATHER && !kpos) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
-  if (!make_tile_map(&mq, q, (uint64_t)dm.b * dm.hq * dm.n, D, kBM) ||
-      !make_tile_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D, kBN) ||
-      !make_tile_map(&mv, vp, (uint64_t)dm.b * dm.hkv * dm.n, D, kBN))
+  if (!make_tile_map(&mq, q, (uint64_t)dm.b * dm.hq * dm.n, D, kBM)) return cudaErrorInvalidValue;
+  if (GATHER) {
+    mk = mq, mv = mq;  // unused: K and V rows are gathered with cp.async
+  } else if (!make_tile_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D, kBN) ||
+             !make_tile_map(&mv, vp, (uint64_t)dm.b * dm.hkv * dm.n, D, kBN)) {
     return cudaErrorInvalidValue;
+  }
   constexpr size_t smem = smem2<D>();
-  cudaError_t e = cudaFuncSetAttribute(attn_tc2_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = attn_tc2_kernel<D, GATHER>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   // The setmaxnreg split above is only safe at the launch allocation it was
   // sized for; with any other count the softmax warps could wait forever.
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, attn_tc2_kernel<D>);
+  e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   const long long total = (long long)dm.b * dm.hq * dm.nb;
   const unsigned grid = (unsigned)((total + 1) / 2);
-  attn_tc2_kernel<D><<<grid, kThreads, smem, st>>>(mq, mk, mv, kpos, qpos, idx, cnt, (bf16 *)out,
-                                                   lse, dm, sigma * kLog2e, err, fault,
-                                                   scatter ? 1 : 0);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, kpos, qpos, idx, cnt, (bf16 *)out, lse, dm,
+                                    sigma * kLog2e, err, fault, scatter ? 1 : 0,
+                                    (const bf16 *)kp, (const bf16 *)vp);
   return cudaGetLastError();
 }
 
@@ -555,10 +661,19 @@ cudaError_t run2(const Dims &dm, const void *q, const void *kp, const void *vp,
 cudaError_t launch_attn_tc2(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                             const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            int fault, bool scatter, cudaStream_t st) {
+                            int fault, bool scatter, bool gather, cudaStream_t st) {
+  if (gather) {
+    if (dm.d == 64)
+      return run2<64, true>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+                            scatter, st);
+    return run2<128, true>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+                           scatter, st);
+  }
   if (dm.d == 64)
-    return run2<64>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, scatter, st);
-  return run2<128>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault, scatter, st);
+    return run2<64, false>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+                           scatter, st);
+  return run2<128, false>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+                          scatter, st);
 }
 
 }  // namespace pbs

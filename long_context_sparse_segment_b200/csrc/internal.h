@@ -49,11 +49,13 @@ cudaError_t launch_select(const Dims &dm, const double *qsum, const double *ksum
                           uint8_t *mask, void *scratch, int *err, cudaStream_t st);
 
 // block-sparse forward; with `scatter` each output row is written at its
-// query's original position (qpos) instead of its place in the given order
+// query's original position (qpos) instead of its place in the given order;
+// with `gather` kp and vp are the natural K and V and key p of the permuted
+// order is read from row kpos[p] (no K', V' copies)
 cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const void *vp,
                         const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                         const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                        bool scatter, cudaStream_t st);
+                        bool scatter, bool gather, cudaStream_t st);
 
 // the forward on the tcgen05 tensor cores (B = 128, d in {64, 128})
 bool attn_tc_supported(const Dims &dm);
@@ -66,13 +68,13 @@ cudaError_t launch_attn_tc(const Dims &dm, const void *q, const void *kp, const 
 cudaError_t launch_attn_tc2(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                             const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            int fault, bool scatter, cudaStream_t st);
+                            int fault, bool scatter, bool gather, cudaStream_t st);
 
 // the same forward on the legacy warp-MMA path
 cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                             const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            bool scatter, cudaStream_t st);
+                            bool scatter, bool gather, cudaStream_t st);
 
 // diagnostics: block attention mass (tcgen05, B = 128, G <= 4), and per row
 // the coverage of a list and the fewest blocks for a target coverage

@@ -113,9 +113,11 @@ __global__ void __launch_bounds__(kGatherThreads)
       src = p;
     }
     const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(k + (row0 + src) * D) + c);
-    const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(v + (row0 + src) * D) + c);
-    reinterpret_cast<uint4 *>(kp + (row0 + p) * D)[c] = kv;
-    reinterpret_cast<uint4 *>(vp + (row0 + p) * D)[c] = vv;
+    if (kp) {  // K', V' written, or only the order and the block sums
+      const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(v + (row0 + src) * D) + c);
+      reinterpret_cast<uint4 *>(kp + (row0 + p) * D)[c] = kv;
+      reinterpret_cast<uint4 *>(vp + (row0 + p) * D)[c] = vv;
+    }
     add_bf16x8(acc, kv);
     if (q) {
       for (int gl = 0; gl < dm.G; ++gl) {

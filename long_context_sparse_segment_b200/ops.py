@@ -64,9 +64,10 @@ def score(q, k, block, segment=None, scale=0.0, ws=None, out=None):
     return imp
 
 
-def permute(imp, k, v, block, segment, q=None, kbar=True, hq=None):
+def permute(imp, k, v, block, segment, q=None, kbar=True, hq=None, materialize=True):
     """Segment-local order and gathers. Returns dict(kpos, k_perm, v_perm,
-    kbar_sum[, q_perm])."""
+    kbar_sum[, q_perm]); without ``materialize`` only the order and the key
+    block sums are produced (k_perm, v_perm None) for attn_fwd_gather."""
     _need(imp, "imp", torch.float32)
     _need(k, "k", torch.bfloat16, imp.device)
     _need(v, "v", torch.bfloat16, imp.device)
@@ -77,8 +78,8 @@ def permute(imp, k, v, block, segment, q=None, kbar=True, hq=None):
     shp = Shape(b, hq or hkv, hkv, n, d, block, segment)
     out = {
         "kpos": torch.empty(b, hkv, n, dtype=torch.int32, device=k.device),
-        "k_perm": torch.empty_like(k),
-        "v_perm": torch.empty_like(v),
+        "k_perm": torch.empty_like(k) if materialize else None,
+        "v_perm": torch.empty_like(v) if materialize else None,
         "kbar_sum": (torch.empty(b, hkv, n // block, d, dtype=torch.float64, device=k.device)
                      if kbar else None),
         "q_perm": torch.empty_like(q) if q is not None else None,
@@ -137,6 +138,29 @@ def attn_fwd(q, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt, block, segment, sc
     return (o, l) if lse else o
 
 
+def attn_fwd_gather(q, k, v, kpos, qpos, blk_idx, blk_cnt, block, segment, scale=0.0,
+                    lse=False, out=None, unpermute=False):
+    """attn_fwd on the natural k, v: key slot p is read from row kpos[p]
+    (pbs_attn_fwd_gather), so no permuted copies are needed. Same result,
+    bit for bit, as attn_fwd on k[kpos], v[kpos]."""
+    _need(q, "q", torch.bfloat16)
+    _need(k, "k", torch.bfloat16, q.device)
+    _need(v, "v", torch.bfloat16, q.device)
+    _need(kpos, "kpos", torch.int32, q.device)
+    if qpos is not None:
+        _need(qpos, "qpos", torch.int32, q.device)
+    _need(blk_idx, "blk_idx", torch.int32, q.device)
+    _need(blk_cnt, "blk_cnt", torch.int32, q.device)
+    shp = shape_of(q, k, block, segment)
+    o = out if out is not None else torch.empty_like(q)
+    l = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if lse else None
+    check(lib().pbs_attn_fwd_gather(_ptr(q), _ptr(k), _ptr(v), _ptr(kpos), _ptr(qpos),
+                                    _ptr(blk_idx), _ptr(blk_cnt), _ptr(o), _ptr(l), shp, scale,
+                                    1 if unpermute else 0, _stream(q.device)),
+          "pbs_attn_fwd_gather")
+    return (o, l) if lse else o
+
+
 def unpermute(o_perm, qpos, hkv, block, segment, out=None):
     """o[b, g, qpos[b, g/G, p]] = o_perm[b, g, p]."""
     _need(o_perm, "o_perm", torch.bfloat16)
@@ -160,19 +184,26 @@ def device_status(device=None, detail=False):
 
 
 def pbs_attention(q, k, v, block, segment, mode="threshold", param=0.9, scale=0.0,
-                  permute_q=False, keep=False, fused_unpermute=True):
+                  permute_q=False, keep=False, fused_unpermute=True, gather_kv=False):
     """The whole prefill path: score -> permute -> select -> attend ->
     unpermute. Returns o [b, hq, n, d] bf16 in the natural query order, or a
     dict with every intermediate when ``keep`` is true. In permuted-query
     mode the last two steps are one call unless ``fused_unpermute`` is
-    false (then ``o_perm`` holds the rows in permuted order)."""
+    false (then ``o_perm`` holds the rows in permuted order). With
+    ``gather_kv`` the permutation writes only the key order and block sums
+    and the forward reads K, V through it (no K', V' copies)."""
     imp = score(q, k, block, segment, scale)
-    perm = permute(imp, k, v, block, segment, q=q if permute_q else None, hq=q.shape[1])
+    perm = permute(imp, k, v, block, segment, q=q if permute_q else None, hq=q.shape[1],
+                   materialize=not gather_kv)
     q_used = perm["q_perm"] if permute_q else q
     qpos = perm["kpos"] if permute_q else None
     idx, cnt, _ = select_blocks(q_used, perm["k_perm"], perm["kbar_sum"], block, segment, mode,
                                 param, scale)
-    if permute_q and fused_unpermute:
+    if gather_kv:
+        o = attn_fwd_gather(q_used, k, v, perm["kpos"], qpos, idx, cnt, block, segment, scale,
+                            unpermute=permute_q)
+        o_perm = None
+    elif permute_q and fused_unpermute:
         o = attn_fwd(q_used, perm["k_perm"], perm["v_perm"], perm["kpos"], qpos, idx, cnt,
                      block, segment, scale, unpermute=True)
         o_perm = None

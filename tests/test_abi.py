@@ -115,6 +115,26 @@ def test_workspace_sizes_grow_with_the_problem(lib):
     assert pbs.workspace_bytes(shape(), _lib.OP_ATTN) == 0
 
 
+def test_gathering_forward_and_order_only_permute_arguments(lib):
+    s = shape()
+    fake = ctypes.c_void_p(1 << 20)
+    other = ctypes.c_void_p(1 << 24)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    # the carried key positions are required
+    assert lib.pbs_attn_fwd_gather(fake, fake, fake, None, None, fake, fake, other, None, s,
+                                   0.0, 0, None) == _lib.ERR_INVALID_ARG
+    assert lib.pbs_attn_fwd_gather(fake, odd, fake, fake, None, fake, fake, other, None, s,
+                                   0.0, 0, None) == _lib.ERR_INVALID_ARG
+    # rows written at qpos must not land on an input still being read
+    assert lib.pbs_attn_fwd_gather(fake, other, other, other, other, other, other, fake, None, s,
+                                   0.0, 1, None) == _lib.ERR_INVALID_ARG
+    # K' and V' are written together or not at all
+    assert lib.pbs_permute(fake, fake, fake, None, other, None, None, fake, None, s,
+                           None) == _lib.ERR_INVALID_ARG
+    assert lib.pbs_permute(fake, fake, fake, None, None, other, None, fake, None, s,
+                           None) == _lib.ERR_INVALID_ARG
+
+
 def test_fused_forward_rejects_output_aliasing_an_input(lib):
     s = shape()
     fake = ctypes.c_void_p(1 << 20)

@@ -131,3 +131,21 @@ def test_llama128k_all_blocks_is_dense_causal(dev):
 def test_stack64k_one_layer_batch2(dev):
     w = WORKLOADS["stack64k"]
     check_full_size(w, dev, heads=[7], blocks=sample_blocks(w.nb, w.segment // w.block), layer=3)
+
+
+@pytest.mark.parametrize("name", ["llama32k", "llama128k"])
+def test_gathering_forward_full_size(name, dev):
+    """At full size the forward that reads K, V through the key order gives
+    the forward on the gathered copies bit for bit, and the order-only
+    permutation the same order and block sums."""
+    w = WORKLOADS[name]
+    B, S = w.block, w.segment
+    q, k, v, res = run_path(w, dev)
+    imp = pbs.score(q, k, B, S)
+    lean = pbs.permute(imp, k, v, B, S, hq=w.hq, materialize=False)
+    assert torch.equal(lean["kpos"], res["kpos"])
+    assert torch.equal(lean["kbar_sum"], res["kbar_sum"])
+    o = pbs.attn_fwd_gather(q, k, v, lean["kpos"], None, res["idx"], res["cnt"], B, S)
+    torch.cuda.synchronize()
+    assert pbs.device_status() == 0
+    assert torch.equal(o, res["o"])
