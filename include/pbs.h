@@ -297,9 +297,16 @@ pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out,
  * library's (the pages do not treat host buffers).
  *
  * The work is split by KV group (batch b, KV head h: query heads
- * h*G .. h*G+G-1): the copy of group i+1 into the device (on `h2d`) and of
- * group i-1 back to the host (on `d2h`) run while group i is computed (on
- * `compute`), in two device slots of the workspace used in turn. Work
+ * h*G .. h*G+G-1), in two device slots of the workspace used in turn, and
+ * inside a group by query head. On `h2d`: K, V and the last query block of
+ * each head (what the scoring and the permutation need), then the query
+ * heads in steps. On `compute`: the group's scoring and permutation, then
+ * per step, as soon as its heads have arrived, their selection and
+ * forward. On `d2h`: each step's output as soon as it is computed. A step
+ * is the fewest query heads (a divisor of G) whose forward still fills the
+ * device (three waves of CTAs): one head at 128K, the whole group at 32K.
+ * So the copies of one group overlap the compute of the previous one, and
+ * only one step's copies are exposed at the start and at the end. Work
  * issued later on `compute` is ordered after the last copy to the host, so
  * synchronising `compute` makes `out` valid. `h2d` and `d2h` may be the same
  * stream (the copies then run one after the other) but must differ from
@@ -312,7 +319,8 @@ pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out,
  *   k, v         host [batch, hkv, n, d] bf16
  *   mode, param  as for pbs_select_blocks
  *   ws           device workspace of pbs_workspace_bytes(s, PBS_OP_HOST_PATH)
- *                bytes (two slots of one KV group's buffers)
+ *                bytes (two slots of one KV group's buffers; the size depends
+ *                on the current device's SM count through the step size)
  * Returns PBS_ERR_UNSUPPORTED when the scoring step does not support the
  * group shape (see pbs_score).
  */

@@ -2,9 +2,11 @@
 // word, and the launches of the five steps. Declared in include/pbs.h.
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
+#include <vector>
 
 #include "../../include/pbs.h"
 #include "common.cuh"
@@ -78,6 +80,31 @@ Dims group_dims(const Dims &dm) {
   return g;
 }
 
+// The host path's unit of selection, forward and copies: `hs` query heads
+// of one KV group, the fewest (a divisor of G) whose forward still fills
+// three waves of two-tile CTAs, so that splitting a group costs no
+// occupancy.
+// PBS_HOST_STEP_HEADS=<k> (a divisor of G) sets the step instead (a
+// diagnostic switch: the tests check that every step size gives the same
+// result).
+int heads_per_step(const Dims &g) {
+  if (const char *env = getenv("PBS_HOST_STEP_HEADS")) {
+    const int k = atoi(env);
+    if (k >= 1 && k <= g.G && g.G % k == 0) return k;
+  }
+  const long long want = 3LL * sm_count();
+  for (int hs = 1; hs < g.G; ++hs)
+    if (g.G % hs == 0 && (long long)hs * ((g.nb + 1) / 2) >= want) return hs;
+  return g.G;
+}
+
+Dims step_dims(const Dims &g, int hs) {
+  Dims h = g;
+  h.hq = hs;
+  h.G = hs;
+  return h;
+}
+
 struct Slot {
   void *q, *k, *v, *kp, *vp, *o, *score_ws;
   float *imp;
@@ -107,7 +134,9 @@ size_t carve_slot(uint8_t *base, const Dims &g, Slot *sl) {
   t.idx = (int32_t *)take((size_t)g.hq * g.nb * g.nb * 4);
   t.cnt = (int32_t *)take((size_t)g.hq * g.nb * 4);
   t.score_ws = take(score_ws_bytes(g));
-  t.qsum = (double *)take(select_ws_bytes(g, false));
+  // the steps of a group are selected one after the other on one stream,
+  // so one step's selection workspace serves them all
+  t.qsum = (double *)take(select_ws_bytes(step_dims(g, heads_per_step(g)), false));
   if (sl) *sl = t;
   return off;
 }
@@ -310,57 +339,84 @@ pbs_status pbs_attention_host(const void *q, const void *k, const void *v, void 
   const size_t slot_bytes = carve_slot(base, g, &slot[0]);
   carve_slot(base + slot_bytes, g, &slot[1]);
 
-  cudaStream_t cs = (cudaStream_t)compute, hs = (cudaStream_t)h2d, ds = (cudaStream_t)d2h;
-  cudaEvent_t ev[3][2] = {};  // [copied in, computed, copied out][slot]
-  for (auto &row : ev)
-    for (auto &e : row)
-      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
-        for (auto &r2 : ev)
-          for (auto &e2 : r2)
-            if (e2) cudaEventDestroy(e2);
-        return PBS_ERR_CUDA;
-      }
+  cudaStream_t cs = (cudaStream_t)compute, hst = (cudaStream_t)h2d, ds = (cudaStream_t)d2h;
+  // per slot: [0] K, V and the last query block of every head copied in,
+  // [1 + st] the query heads of step st copied in, [1 + steps + st] step st
+  // computed, [1 + 2 steps] the slot's last output copied out
+  const int G = dm.G, hs = heads_per_step(g), steps = G / hs, per_slot = 2 + 2 * steps;
+  std::vector<cudaEvent_t> evs(2 * (size_t)per_slot, nullptr);
+  cudaError_t e = cudaSuccess;
+  for (auto &x : evs)
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    for (auto &x : evs)
+      if (x) cudaEventDestroy(x);
+    return PBS_ERR_CUDA;
+  }
+  auto ev = [&](int sid, int k) { return evs[(size_t)sid * per_slot + k]; };
+  const Dims h1 = step_dims(g, hs);
   int *err = error_word();
   const float sigma_f = (float)resolve_sigma(scale, dm.d);
   const double sigma_d = resolve_sigma(scale, dm.d);
-  const size_t qb = (size_t)g.hq * g.n * g.d * 2, kb = (size_t)g.n * g.d * 2;
+  const size_t hb = (size_t)g.n * g.d * 2;  // one head's rows (Q, O, K or V)
+  const size_t lastb = (size_t)g.B * g.d * 2, restb = hb - lastb;
+  const size_t nb = (size_t)g.nb;
   const int groups = dm.b * dm.hkv;
-  cudaError_t e = cudaSuccess;
+  auto at = [](const void *p, size_t off) { return (const uint8_t *)p + off; };
   for (int i = 0; i < groups && e == cudaSuccess; ++i) {
     const int sid = i & 1, bi = i / dm.hkv, h = i % dm.hkv;
     const Slot &sl = slot[sid];
-    const size_t qoff = ((size_t)bi * dm.hq + (size_t)h * dm.G) * qb / g.hq;
-    const size_t koff = ((size_t)bi * dm.hkv + h) * kb;
-    // in: the slot is free once group i - 2 has been copied out
-    if (i >= 2) e = cudaStreamWaitEvent(hs, ev[2][sid], 0);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(sl.q, (const uint8_t *)q + qoff, qb, cudaMemcpyHostToDevice, hs);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(sl.k, (const uint8_t *)k + koff, kb, cudaMemcpyHostToDevice, hs);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(sl.v, (const uint8_t *)v + koff, kb, cudaMemcpyHostToDevice, hs);
-    if (e == cudaSuccess) e = cudaEventRecord(ev[0][sid], hs);
-    // the five steps on the group
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev[0][sid], 0);
+    const size_t qoff = ((size_t)bi * dm.hq + (size_t)h * G) * hb;  // head h*G of batch bi
+    const size_t koff = ((size_t)bi * dm.hkv + h) * hb;
+    uint8_t *sq = (uint8_t *)sl.q, *so = (uint8_t *)sl.o;
+    // in: the slot is free once group i - 2 has been copied out. First what
+    // the scoring and the permutation need (K, V, the last query block of
+    // each head), then the query heads one by one
+    if (i >= 2) e = cudaStreamWaitEvent(hst, ev(sid, 1 + 2 * steps), 0);
+    for (int gl = 0; gl < G && e == cudaSuccess; ++gl)
+      e = cudaMemcpyAsync(sq + gl * hb + restb, at(q, qoff + gl * hb + restb), lastb,
+                          cudaMemcpyHostToDevice, hst);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sl.k, at(k, koff), hb, cudaMemcpyHostToDevice, hst);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sl.v, at(v, koff), hb, cudaMemcpyHostToDevice, hst);
+    if (e == cudaSuccess) e = cudaEventRecord(ev(sid, 0), hst);
+    for (int st = 0; st < steps && e == cudaSuccess; ++st) {
+      for (int gl = st * hs; gl < (st + 1) * hs && e == cudaSuccess && restb; ++gl)
+        e = cudaMemcpyAsync(sq + gl * hb, at(q, qoff + gl * hb), restb, cudaMemcpyHostToDevice,
+                            hst);
+      if (e == cudaSuccess) e = cudaEventRecord(ev(sid, 1 + st), hst);
+    }
+    // the group's scoring and permutation
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev(sid, 0), 0);
     if (e == cudaSuccess) e = launch_score(g, sl.q, sl.k, sl.imp, sigma_f, sl.score_ws, err, cs);
     if (e == cudaSuccess) e = launch_segsort(g, sl.imp, sl.kpos, err, cs);
     if (e == cudaSuccess)
       e = launch_gather(g, sl.kpos, sl.k, sl.v, nullptr, sl.kp, sl.vp, nullptr, sl.kbar, err, cs);
-    if (e == cudaSuccess && scored) e = launch_blocksum(g, g.hq, sl.q, sl.qsum, cs);
-    if (e == cudaSuccess)
-      e = launch_select(g, sl.qsum, sl.kbar, mode, param, sigma_d, sl.idx, sl.cnt, nullptr,
-                        (uint8_t *)sl.qsum + select_qsum_bytes(g), err, cs);
-    if (e == cudaSuccess)
-      e = launch_attn(g, sl.q, sl.kp, sl.vp, sl.kpos, nullptr, sl.idx, sl.cnt, sl.o, nullptr,
-                      sigma_f, err, false, false, cs);
-    if (e == cudaSuccess) e = cudaEventRecord(ev[1][sid], cs);
-    // out
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(ds, ev[1][sid], 0);
-    if (e == cudaSuccess) e = cudaMemcpyAsync((uint8_t *)out + qoff, sl.o, qb, cudaMemcpyDeviceToHost, ds);
-    if (e == cudaSuccess) e = cudaEventRecord(ev[2][sid], ds);
+    // then per step of hs query heads, as they arrive: selection, forward,
+    // copy out
+    for (int st = 0; st < steps && e == cudaSuccess; ++st) {
+      const int gl = st * hs;
+      const uint8_t *qh = sq + gl * hb;
+      int32_t *idx = sl.idx + (size_t)gl * nb * nb, *cnt = sl.cnt + (size_t)gl * nb;
+      e = cudaStreamWaitEvent(cs, ev(sid, 1 + st), 0);
+      if (e == cudaSuccess && scored) e = launch_blocksum(h1, hs, qh, sl.qsum, cs);
+      if (e == cudaSuccess)
+        e = launch_select(h1, sl.qsum, sl.kbar, mode, param, sigma_d, idx, cnt, nullptr,
+                          (uint8_t *)sl.qsum + select_qsum_bytes(h1), err, cs);
+      if (e == cudaSuccess)
+        e = launch_attn(h1, qh, sl.kp, sl.vp, sl.kpos, nullptr, idx, cnt, so + gl * hb, nullptr,
+                        sigma_f, err, false, false, cs);
+      if (e == cudaSuccess) e = cudaEventRecord(ev(sid, 1 + steps + st), cs);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(ds, ev(sid, 1 + steps + st), 0);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync((uint8_t *)out + qoff + gl * hb, so + gl * hb, hs * hb,
+                            cudaMemcpyDeviceToHost, ds);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev(sid, 1 + 2 * steps), ds);
   }
   // work queued on the copy streams is ordered before later work on `compute`
   for (int sid = 0; sid < 2 && sid < groups && e == cudaSuccess; ++sid)
-    e = cudaStreamWaitEvent(cs, ev[2][sid], 0);
-  for (auto &row : ev)
-    for (auto &ee : row) cudaEventDestroy(ee);  // released once their work completes
+    e = cudaStreamWaitEvent(cs, ev(sid, 1 + 2 * steps), 0);
+  for (auto &x : evs) cudaEventDestroy(x);  // released once their work completes
   return cuda_status(e);
 }
 

@@ -38,6 +38,9 @@ cudaError_t launch_gather(const Dims &dm, const int32_t *kpos, const void *k, co
 cudaError_t launch_blocksum(const Dims &dm, int heads, const void *x, double *out,
                             cudaStream_t st);
 
+// SMs of the current device (148 when the query fails)
+int sm_count();
+
 // block lists from pooled sums
 // workspace: pooled query sums [+ pooled key sums] + scratch (score keys and
 // softmax weights per (batch, query head, query block, key block))

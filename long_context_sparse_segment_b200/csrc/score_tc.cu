@@ -373,16 +373,6 @@ __global__ void score_tc_combine(const float2 *__restrict__ partial, float *__re
   off[i] = M + log2f(L);
 }
 
-int sm_count() {
-  int dev = 0, c = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) {
-    cudaGetLastError();
-    return 148;
-  }
-  return c;
-}
-
 // CTAs per (batch, KV head): one wave over the SMs, at most one per tile.
 int tc_splits(const Dims &dm) {
   const int bh = dm.b * dm.hkv;
@@ -424,6 +414,16 @@ cudaError_t run_tc(const Dims &dm, const void *q, const void *k, float *imp, flo
 }
 
 }  // namespace
+
+int sm_count() {
+  int dev = 0, c = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return c;
+}
 
 bool score_tc_supported(const Dims &dm) {
   const int R = dm.G * dm.B;

@@ -361,3 +361,26 @@ def test_host_buffer_path_many_groups_reuse_both_slots(dev):
     torch.cuda.synchronize()
     assert pbs.device_status() == 0
     assert_outputs_close(f64(o_host), f64(o_dev), "host vs device path")
+
+
+@pytest.mark.parametrize("name", ["gqa2k", "d128_b64", "groups8"])
+def test_host_buffer_path_steps_of_query_heads(name, dev, monkeypatch):
+    """The host path streams each KV group's query heads in steps (selection,
+    forward and copies per step). Every step size gives the same output bit
+    for bit: a query head's lists and rows do not depend on which heads share
+    its launch."""
+    w = CASES.get(name) or Workload("groups8", 2, 8, 4, 1024, 128, 128, 256, "topk_frac", 0.5,
+                                    "uniform", 0.05, seed=11)
+    q, k, v, _ = make_inputs(w)
+    q, k, v = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    outs = {}
+    for step in (w.group, 2, 1):
+        if w.group % step:
+            continue
+        monkeypatch.setenv("PBS_HOST_STEP_HEADS", str(step))
+        o = pbs.attention_host(q, k, v, w.block, w.segment, w.mode, w.param)
+        torch.cuda.synchronize()  # the output is valid once the stream has synchronised
+        assert pbs.device_status() == 0
+        outs[step] = o.clone()
+    for step, o in outs.items():
+        assert torch.equal(o, outs[w.group]), f"step of {step} heads"
