@@ -37,7 +37,7 @@ from long_context_sparse_segment_b200.workloads import WORKLOADS, make_inputs  #
 
 METRIC = "PBS-Attn prefill ms and effective TFLOP/s (% BF16 peak) at N=32K–128K vs dense"
 UNIT = "TFLOP/s"
-LAUNCHES_PER_LAYER = 8  # score 3, permute 2, select 2, forward 1
+LAUNCHES_PER_LAYER = 9  # score 3, permute 2, select 3 (pooling, scores, lists), forward 1
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
