@@ -96,15 +96,20 @@ __device__ __forceinline__ Tile make_tile(int item, int total, const Dims &dm,
                                           const int32_t *blk_idx, const int32_t *blk_cnt,
                                           int *err) {
   Tile t;
-  const int heads = dm.b * dm.hq;
   if (item >= total) {
     t.bg = 0, t.I = 0, t.bh = 0, t.count = 0, t.segI = 0, t.list = blk_idx;
     return t;
   }
-  t.I = dm.nb - 1 - item / heads;  // heavy query blocks first
-  t.bg = item % heads;
-  const int b = t.bg / dm.hq, g = t.bg % dm.hq;
-  t.bh = b * dm.hkv + g / dm.G;
+  // KV groups one after the other, so that the K'/V' tiles in use at a time
+  // are one KV head's (L2-resident reuse across the group's query heads
+  // and neighbouring query blocks); inside a group heavy query blocks first,
+  // the G query heads of a block adjacent (a CTA's two tiles share a block
+  // index whenever G is even)
+  const int per_group = dm.G * dm.nb;
+  const int r = item % per_group;
+  t.bh = item / per_group;
+  t.I = dm.nb - 1 - r / dm.G;
+  t.bg = (t.bh / dm.hkv) * dm.hq + (t.bh % dm.hkv) * dm.G + r % dm.G;
   t.segI = t.I / dm.spb;
   t.list = blk_idx + ((size_t)t.bg * dm.nb + t.I) * dm.nb;
   t.count = blk_cnt[(size_t)t.bg * dm.nb + t.I];
