@@ -53,6 +53,10 @@ def parse():
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N > 1: every rank runs the whole workload (weak scaling), or "
                          "the KV groups of one workload are split over the ranks (strong)")
+    ap.add_argument("--queries", choices=["natural", "fused", "separate"], default="natural",
+                    help="natural query order (the default path), or queries permuted with "
+                         "the keys and the inverse permutation fused into the forward's "
+                         "epilogue or run as its own step")
     ap.add_argument("--gather-kv", action="store_true",
                     help="the forward reads K, V through the key order (pbs_attn_fwd_gather); "
                          "the permutation writes only the order and block sums")
@@ -162,18 +166,23 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- GPU arm
 class Layer:
-    def __init__(self, w, dev, layer, seed_offset, gather_kv=False):
+    def __init__(self, w, dev, layer, seed_offset, gather_kv=False, queries="natural"):
         self.w = w
         self.gather_kv = gather_kv  # the forward reads K, V through the key order
+        # "natural", or permuted queries with the inverse permutation "fused"
+        # into the forward or run as its own step ("separate")
+        self.queries = queries
         self.q, self.k, self.v, _ = make_inputs(w, dev, layer=layer, seed=w.seed + layer + seed_offset)
         self.out = None
+        self.o_perm = None
 
 
 def run_layer(layer, ev=None):
     """The five steps on one layer; returns (o, blk_cnt). ev: dict of event
-    pairs recorded around score / permute / select / forward."""
+    pairs recorded around score / permute / select / forward / unpermute."""
     w = layer.w
     B, S = w.block, w.segment
+    permuted_q = layer.queries != "natural"
 
     def mark(name, i):
         if ev is not None:
@@ -183,20 +192,31 @@ def run_layer(layer, ev=None):
     imp = pbs.score(layer.q, layer.k, B, S)
     mark("score", 1)
     mark("permute", 0)
-    perm = pbs.permute(imp, layer.k, layer.v, B, S, hq=w.hq, materialize=not layer.gather_kv)
+    perm = pbs.permute(imp, layer.k, layer.v, B, S, q=layer.q if permuted_q else None, hq=w.hq,
+                       materialize=not layer.gather_kv)
     mark("permute", 1)
+    q_used = perm["q_perm"] if permuted_q else layer.q
+    qpos = perm["kpos"] if permuted_q else None
     mark("select", 0)
-    idx, cnt, _ = pbs.select_blocks(layer.q, perm["k_perm"], perm["kbar_sum"], B, S, w.mode,
+    idx, cnt, _ = pbs.select_blocks(q_used, perm["k_perm"], perm["kbar_sum"], B, S, w.mode,
                                     w.param)
     mark("select", 1)
+    fused = layer.queries == "fused"
     mark("attn", 0)
     if layer.gather_kv:
-        o = pbs.attn_fwd_gather(layer.q, layer.k, layer.v, perm["kpos"], None, idx, cnt, B, S,
-                                out=layer.out)
+        o = pbs.attn_fwd_gather(q_used, layer.k, layer.v, perm["kpos"], qpos, idx, cnt, B, S,
+                                out=layer.o_perm if layer.queries == "separate" else layer.out,
+                                unpermute=fused)
     else:
-        o = pbs.attn_fwd(layer.q, perm["k_perm"], perm["v_perm"], perm["kpos"], None, idx, cnt,
-                         B, S, out=layer.out)
+        fwd_out = layer.o_perm if layer.queries == "separate" else layer.out
+        o = pbs.attn_fwd(q_used, perm["k_perm"], perm["v_perm"], perm["kpos"], qpos, idx, cnt,
+                         B, S, out=fwd_out, unpermute=fused)
     mark("attn", 1)
+    mark("unpermute", 0)
+    if layer.queries == "separate":
+        layer.o_perm = o
+        o = pbs.unpermute(o, qpos, w.hkv, B, S, out=layer.out)
+    mark("unpermute", 1)
     layer.out = o
     return o, cnt
 
@@ -274,8 +294,8 @@ def gpu_arm(args):
         seed_offset = first
     else:
         seed_offset = rank_seed_offset(rank)
-    layers = [Layer(w, dev, l, seed_offset=seed_offset, gather_kv=args.gather_kv)
-              for l in range(w.layers)]
+    layers = [Layer(w, dev, l, seed_offset=seed_offset, gather_kv=args.gather_kv,
+                    queries=args.queries) for l in range(w.layers)]
     torch.cuda.synchronize()
 
     # warm-up (also fixes the kept-block counts of this input)
@@ -286,7 +306,7 @@ def gpu_arm(args):
             total_blocks += float(cnt.sum().item())
     flops_per_step = block_flops(w, total_blocks)
 
-    names = ("score", "permute", "select", "attn")
+    names = ("score", "permute", "select", "attn", "unpermute")
     evs = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for n in names} for _ in range(args.steps * len(layers))]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -331,7 +351,10 @@ def gpu_arm(args):
                    "d": w.d, "block": w.block, "segment": w.segment, "layers": w.layers,
                    "selection": f"{w.mode} {w.param}", "l2": "inputs larger than L2",
                    "parallelism": f"heads/{world}" if sharded else f"replicas x{world}",
-                   "kv": "gathered inside the forward" if args.gather_kv else "permuted copies"},
+                   "kv": "gathered inside the forward" if args.gather_kv else "permuted copies",
+                   "queries": {"natural": "natural order",
+                               "fused": "permuted, inverse fused into the forward",
+                               "separate": "permuted, inverse as its own step"}[args.queries]},
         "density": round(total_blocks / (len(layers) * w.batch * w.hq * w.nb * (w.nb + 1) / 2), 4),
         "breakdown_ms": {n: round(v, 4) for n, v in per.items()},
         "dense_attn_ms": round(dense_ms * len(layers), 4),
@@ -340,7 +363,8 @@ def gpu_arm(args):
         "clocks": clock_info,
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "ms_per_step": round(e2e_ms, 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": LAUNCHES_PER_LAYER * len(layers) * args.steps,
+        "gpu_launches": (LAUNCHES_PER_LAYER + (args.queries == "separate")) * len(layers)
+                        * args.steps,
         "roofline": {"kernel": "pbs_attn_fwd", "bound": "tensor",
                      "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peak, 4), "peak_kind":
