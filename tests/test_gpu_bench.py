@@ -1,0 +1,73 @@
+"""bench.py on the GPU: every timed mode computes the path's result, and the
+JSON line carries the fields of its contract."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+
+import long_context_sparse_segment_b200 as pbs
+from long_context_sparse_segment_b200.workloads import WORKLOADS, Workload
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    return torch.device("cuda", 0)
+
+
+@pytest.mark.parametrize("queries", ["natural", "fused", "separate"])
+@pytest.mark.parametrize("gather_kv", [False, True])
+def test_timed_step_computes_the_path(queries, gather_kv, dev):
+    """The step bench.py times gives, in every mode, the output of the
+    path's own entry point in the matching query mode."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    w = Workload("bench2k", 1, 8, 2, 2048, 128, 128, 512, "topk_frac", 0.3, "per_segment", 0.02)
+    layer = bench.Layer(w, dev, 0, seed_offset=0, gather_kv=gather_kv, queries=queries)
+    for _ in range(2):  # the second step reuses the first one's buffers
+        o, cnt = bench.run_layer(layer)
+    torch.cuda.synchronize()
+    assert pbs.device_status() == 0
+    ref = pbs.pbs_attention(layer.q, layer.k, layer.v, w.block, w.segment, w.mode, w.param,
+                            permute_q=queries != "natural")
+    assert torch.equal(o, ref)
+    assert int(cnt.sum()) > 0
+
+
+def run_bench(*args, timeout=600):
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                         capture_output=True, text=True, timeout=timeout)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, res.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+def test_bench_line_contract(dev):
+    d = run_bench("--config", "llama8k", "--steps", "2", "--warmup", "3", "--no-cpu-baseline",
+                  "--e2e-steps", "1")
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "roofline", "e2e", "clocks", "gpu_launches"):
+        assert key in d, key
+    assert d["n_gpus"] == 1 and d["steps"] == 2 and d["warmup"] >= 3
+    assert d["value"] > 0 and d["ms_per_step"] > 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "llama8k"
+    assert d["gpu_launches"] == 9 * 2
+    r = d["roofline"]
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert 0 < r["frac"] == pytest.approx(r["achieved"] / r["peak"], rel=1e-3)
+    e = d["e2e"]
+    w = WORKLOADS["llama8k"]
+    assert e["value"] > 0
+    assert e["h2d_bytes_per_step"] == 2 * w.batch * (w.hq + 2 * w.hkv) * w.n * w.d
+    assert e["d2h_bytes_per_step"] == 2 * w.batch * w.hq * w.n * w.d
