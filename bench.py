@@ -57,6 +57,9 @@ def parse():
                     help="natural query order (the default path), or queries permuted with "
                          "the keys and the inverse permutation fused into the forward's "
                          "epilogue or run as its own step")
+    ap.add_argument("--gather-output", action="store_true",
+                    help="with --shard heads on N > 1 GPUs: all-gather every rank's output "
+                         "heads into the whole output on every rank, inside the timed step")
     ap.add_argument("--gather-kv", action="store_true",
                     help="the forward reads K, V through the key order (pbs_attn_fwd_gather); "
                          "the permutation writes only the order and block sums")
@@ -89,6 +92,22 @@ def shard_heads(w, rank, world):
         raise ValueError(f"{w.hkv} KV heads do not split over {world} ranks")
     per = w.hkv // world
     return w.with_(hkv=per, hq=per * w.group), rank * per
+
+
+def gather_heads(o_local, dist, world, out=None):
+    """With the KV groups split over the ranks, each rank holds the output of
+    its own query heads, [b, hq / world, n, d]; this all-gathers them into
+    the whole output [b, hq, n, d] on every rank (one collective, NCCL over
+    NVLink on GPUs; gloo on the CPU in the tests). Rank r's heads come r-th,
+    as shard_heads assigns them."""
+    b, h, n, d = o_local.shape
+    parts = torch.empty((world * b, h, n, d), dtype=o_local.dtype, device=o_local.device)
+    dist.all_gather_into_tensor(parts, o_local.contiguous())  # rank r's slice r-th
+    full = parts.view(world, b, h, n, d).permute(1, 0, 2, 3, 4).reshape(b, world * h, n, d)
+    if out is not None:
+        out.copy_(full)
+        return out
+    return full
 
 
 def job_throughput(flops_rank, ms_rank, dist=None, device="cpu"):
@@ -298,15 +317,27 @@ def gpu_arm(args):
                     queries=args.queries) for l in range(w.layers)]
     torch.cuda.synchronize()
 
+    gathering = args.gather_output and sharded
+
+    def step_layer(L, ev=None):
+        o, cnt = run_layer(L, ev)
+        if ev is not None:
+            ev["gather"][0].record()
+        if gathering:  # the whole output on every rank
+            gather_heads(o, dist, world)
+        if ev is not None:
+            ev["gather"][1].record()
+        return o, cnt
+
     # warm-up (also fixes the kept-block counts of this input)
     for _ in range(max(3, args.warmup)):
         total_blocks = 0.0
         for L in layers:
-            _, cnt = run_layer(L)
+            _, cnt = step_layer(L)
             total_blocks += float(cnt.sum().item())
     flops_per_step = block_flops(w, total_blocks)
 
-    names = ("score", "permute", "select", "attn", "unpermute")
+    names = ("score", "permute", "select", "attn", "unpermute", "gather")
     evs = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for n in names} for _ in range(args.steps * len(layers))]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -318,7 +349,7 @@ def gpu_arm(args):
     i = 0
     for _ in range(args.steps):
         for L in layers:
-            run_layer(L, evs[i])
+            step_layer(L, evs[i])
             i += 1
     stop.record()
     torch.cuda.synchronize()
@@ -350,7 +381,8 @@ def gpu_arm(args):
                    "n": w.n,
                    "d": w.d, "block": w.block, "segment": w.segment, "layers": w.layers,
                    "selection": f"{w.mode} {w.param}", "l2": "inputs larger than L2",
-                   "parallelism": f"heads/{world}" if sharded else f"replicas x{world}",
+                   "parallelism": (f"heads/{world}" + (" + all-gather of O" if gathering else ""))
+                   if sharded else f"replicas x{world}",
                    "kv": "gathered inside the forward" if args.gather_kv else "permuted copies",
                    "queries": {"natural": "natural order",
                                "fused": "permuted, inverse fused into the forward",

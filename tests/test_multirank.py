@@ -124,3 +124,49 @@ def test_two_ranks_head_sharded_throughput_counts_the_sequence_once():
         assert total == pytest.approx(1e12)      # the sequence's flops, once
         assert ms == 6.0                         # the slower rank
         assert value == pytest.approx(1e12 / 6e-3 / 1e12)
+
+
+def _gather_worker(rank, world, port, out):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    from long_context_sparse_segment_b200.workloads import WORKLOADS
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        ok = []
+        for batch in (1, 2):
+            w = WORKLOADS["llama8k"].with_(batch=batch, n=256)
+            ws, first = bench.shard_heads(w, rank, world)
+            # a stand-in for the whole output whose every element names its place
+            full = torch.arange(batch * w.hq * w.n * 8, dtype=torch.float32).reshape(
+                batch, w.hq, w.n, 8)
+            mine = full[:, first * w.group:(first + ws.hkv) * w.group].clone()
+            got = bench.gather_heads(mine, dist, world)
+            ok.append(bool(torch.equal(got, full)))
+            into = torch.empty_like(full)
+            ok.append(bench.gather_heads(mine, dist, world, out=into) is into
+                      and bool(torch.equal(into, full)))
+        out.put((rank, ok))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_all_gather_of_sharded_output_heads():
+    """With --shard heads --gather-output every rank ends with the whole
+    output: the ranks' head slices all-gathered in shard order."""
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = [out.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ok in results:
+        assert all(ok), (rank, ok)
