@@ -57,9 +57,11 @@ def parse():
                     help="natural query order (the default path), or queries permuted with "
                          "the keys and the inverse permutation fused into the forward's "
                          "epilogue or run as its own step")
-    ap.add_argument("--gather-output", action="store_true",
-                    help="with --shard heads on N > 1 GPUs: all-gather every rank's output "
-                         "heads into the whole output on every rank, inside the timed step")
+    ap.add_argument("--gather-output", choices=["none", "nccl", "fused"], default="none",
+                    help="with --shard heads on N > 1 GPUs: the whole output on every rank, "
+                         "inside the timed step, by an NCCL all-gather after the forward or "
+                         "by the forward itself writing into every rank's buffer "
+                         "(pbs_attn_fwd_bcast over symmetric memory)")
     ap.add_argument("--gather-kv", action="store_true",
                     help="the forward reads K, V through the key order (pbs_attn_fwd_gather); "
                          "the permutation writes only the order and block sums")
@@ -194,6 +196,9 @@ class Layer:
         self.q, self.k, self.v, _ = make_inputs(w, dev, layer=layer, seed=w.seed + layer + seed_offset)
         self.out = None
         self.o_perm = None
+        # (output buffers of every rank, this rank's index, first head): the
+        # forward writes its heads into all of them (pbs_attn_fwd_bcast)
+        self.bcast = None
 
 
 def run_layer(layer, ev=None):
@@ -222,7 +227,12 @@ def run_layer(layer, ev=None):
     mark("select", 1)
     fused = layer.queries == "fused"
     mark("attn", 0)
-    if layer.gather_kv:
+    if layer.bcast is not None:
+        outs, me, first_head = layer.bcast
+        pbs.attn_fwd_bcast(q_used, perm["k_perm"], perm["v_perm"], perm["kpos"], idx, cnt, B, S,
+                           outs, head_offset=first_head)
+        o = outs[me]
+    elif layer.gather_kv:
         o = pbs.attn_fwd_gather(q_used, layer.k, layer.v, perm["kpos"], qpos, idx, cnt, B, S,
                                 out=layer.o_perm if layer.queries == "separate" else layer.out,
                                 unpermute=fused)
@@ -317,14 +327,30 @@ def gpu_arm(args):
                     queries=args.queries) for l in range(w.layers)]
     torch.cuda.synchronize()
 
-    gathering = args.gather_output and sharded
+    gathering = args.gather_output if sharded else "none"
+    if gathering == "fused":
+        # every rank's whole-output buffer, mapped into every rank (symmetric
+        # memory: plain peer stores, no multicast); each rank's forward
+        # writes its heads into all of them
+        if args.queries != "natural" or args.gather_kv:
+            raise SystemExit("--gather-output fused runs the natural-order path only")
+        import torch.distributed._symmetric_memory as symm_mem
+        shape = (w_full.batch, w_full.hq, w_full.n, w_full.d)
+        mine = symm_mem.empty(shape, dtype=torch.bfloat16, device=dev)
+        hdl = symm_mem.rendezvous(mine, dist.group.WORLD.group_name)
+        peers = [hdl.get_buffer(r, shape, torch.bfloat16) for r in range(world)]
+        for L in layers:
+            L.bcast = (peers, rank, first * w.group)
+        step_done = torch.zeros(1, device=dev)
 
     def step_layer(L, ev=None):
         o, cnt = run_layer(L, ev)
         if ev is not None:
             ev["gather"][0].record()
-        if gathering:  # the whole output on every rank
+        if gathering == "nccl":  # the whole output on every rank
             gather_heads(o, dist, world)
+        elif gathering == "fused":  # every rank's stores have landed
+            dist.all_reduce(step_done)
         if ev is not None:
             ev["gather"][1].record()
         return o, cnt
@@ -381,7 +407,9 @@ def gpu_arm(args):
                    "n": w.n,
                    "d": w.d, "block": w.block, "segment": w.segment, "layers": w.layers,
                    "selection": f"{w.mode} {w.param}", "l2": "inputs larger than L2",
-                   "parallelism": (f"heads/{world}" + (" + all-gather of O" if gathering else ""))
+                   "parallelism": (f"heads/{world}" + {"none": "", "nccl": " + NCCL all-gather of O",
+                                                        "fused": " + O written to every rank by "
+                                                                 "the forward"}[gathering])
                    if sharded else f"replicas x{world}",
                    "kv": "gathered inside the forward" if args.gather_kv else "permuted copies",
                    "queries": {"natural": "natural order",

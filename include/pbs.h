@@ -12,6 +12,8 @@
  *   pbs_unpermute      inverse permutation of the output rows
  *   pbs_attn_fwd_unpermute  the last two fused: rows written in place
  *   pbs_attn_fwd_gather     the forward reading K, V through kpos (no K', V')
+ *   pbs_attn_fwd_bcast      the forward writing its rows into several
+ *                      buffers (the all-gather of a head-sharded output)
  *   pbs_attention_host the whole path on host buffers, copies overlapped
  *   pbs_block_mass, pbs_coverage  diagnostics: attention coverage and
  *                      block-level density
@@ -273,6 +275,38 @@ pbs_status pbs_attn_fwd_gather(const void *q_or_qperm, const void *k,
                                const int32_t *blk_cnt, void *out, float *lse,
                                pbs_shape s, float scale, int unpermute,
                                pbs_stream_t st);
+
+/*
+ * pbs_attn_fwd_bcast - pbs_attn_fwd (natural query order) whose epilogue
+ * writes every output row into n_out buffers at once: the rows of query
+ * head g of this call go to head head_offset + g of each buffer. With the
+ * KV groups of a sequence split over GPUs, each GPU passes its own output
+ * buffer and its peers' (mapped into this device's address space, e.g. a
+ * symmetric allocation), and head_offset = its first query head: the
+ * forward then also performs the all-gather of the output, its stores to
+ * the peers overlapping the rest of its work. Source: as for pbs_attn_fwd;
+ * the head-sharded runs follow the pages' tensor-parallel setting (the
+ * gist.science summary's experiments at 256K/512K); writing the gathered
+ * output from the forward is this library's.
+ *
+ *   q, k_perm, v_perm, kpos, blk_idx, blk_cnt  as for pbs_attn_fwd (s.hq
+ *                   query heads of this call)
+ *   outs            HOST array of n_out (1..8) device pointers, each to a
+ *                   [batch, hq_total, n, d] bf16 buffer, 16-byte aligned; the
+ *                   call only stores to them (heads head_offset ..
+ *                   head_offset + s.hq - 1); none may be q, k_perm or v_perm
+ *   hq_total        heads of the buffers, >= head_offset + s.hq
+ *   head_offset     first head this call writes, >= 0
+ * The caller orders the readers after the call on every device that writes
+ * into a buffer (e.g. a collective barrier on the same stream).
+ * PBS_ERR_UNSUPPORTED unless B = 128 (the two-tile tcgen05 forward).
+ */
+pbs_status pbs_attn_fwd_bcast(const void *q, const void *k_perm,
+                              const void *v_perm, const int32_t *kpos,
+                              const int32_t *blk_idx, const int32_t *blk_cnt,
+                              void *const *outs, int n_out, int hq_total,
+                              int head_offset, pbs_shape s, float scale,
+                              pbs_stream_t st);
 
 /*
  * pbs_unpermute - inverse permutation of the output rows.

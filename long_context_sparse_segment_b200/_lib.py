@@ -18,7 +18,7 @@ OP_SCORE, OP_PERMUTE, OP_SELECT, OP_ATTN, OP_UNPERMUTE, OP_HOST_PATH = range(6)
 # every entry point declared in include/pbs.h
 EXPORTS = ("pbs_workspace_bytes", "pbs_score", "pbs_score_static", "pbs_permute",
            "pbs_select_blocks", "pbs_attn_fwd", "pbs_unpermute", "pbs_attn_fwd_unpermute",
-           "pbs_attn_fwd_gather", "pbs_attention_host", "pbs_block_mass", "pbs_coverage", "pbs_get_device_status",
+           "pbs_attn_fwd_gather", "pbs_attn_fwd_bcast", "pbs_attention_host", "pbs_block_mass", "pbs_coverage", "pbs_get_device_status",
            "pbs_status_string", "pbs_version")
 
 
@@ -46,6 +46,8 @@ _SIGS = {
     "pbs_attn_fwd_unpermute": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, Shape, _f, _vp]),
     "pbs_attn_fwd_gather": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, Shape, _f, _i,
                                  _vp]),
+    "pbs_attn_fwd_bcast": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(_vp), _i, _i, _i,
+                                Shape, _f, _vp]),
     "pbs_block_mass": (_i, [_vp, _vp, _vp, _vp, Shape, _f, _vp]),
     "pbs_coverage": (_i, [_vp, _vp, _vp, ctypes.c_double, _vp, _vp, Shape, _vp]),
     "pbs_attention_host": (_i, [_vp, _vp, _vp, _vp, Shape, _i, _f, _f, _vp, _sz,

@@ -300,6 +300,37 @@ pbs_status pbs_attn_fwd_gather(const void *q_or_qperm, const void *k, const void
                   unpermute != 0, true, st);
 }
 
+pbs_status pbs_attn_fwd_bcast(const void *q, const void *k_perm, const void *v_perm,
+                              const int32_t *kpos, const int32_t *blk_idx,
+                              const int32_t *blk_cnt, void *const *outs, int n_out,
+                              int hq_total, int head_offset, pbs_shape s, float scale,
+                              pbs_stream_t st) {
+  Dims dm;
+  pbs_status r = check_shape(s, &dm);
+  if (r != PBS_OK) return r;
+  if (!outs || n_out < 1 || n_out > kMaxOuts || head_offset < 0 ||
+      (long long)head_offset + dm.hq > hq_total)
+    return PBS_ERR_INVALID_ARG;
+  if (empty(dm)) return PBS_OK;
+  if (!q || !k_perm || !v_perm || !blk_idx || !blk_cnt || !aligned16(q) || !aligned16(k_perm) ||
+      !aligned16(v_perm) || (kpos && !aligned16(kpos)) || ((uintptr_t)blk_idx & 3u) ||
+      ((uintptr_t)blk_cnt & 3u))
+    return PBS_ERR_INVALID_ARG;
+  OutSet set{};
+  for (int i = 0; i < n_out; ++i) {
+    if (!outs[i] || !aligned16(outs[i]) || outs[i] == q || outs[i] == k_perm ||
+        outs[i] == v_perm)
+      return PBS_ERR_INVALID_ARG;
+    set.p[i] = outs[i];
+  }
+  set.n = n_out, set.hq_total = hq_total, set.head_offset = head_offset;
+  if (!attn_tc_supported(dm)) return PBS_ERR_UNSUPPORTED;
+  const float sigma = (float)resolve_sigma(scale, dm.d);
+  const cudaError_t e = launch_attn_bcast(dm, q, k_perm, v_perm, kpos, blk_idx, blk_cnt, set,
+                                          sigma, error_word(), (cudaStream_t)st);
+  return e == cudaErrorNotSupported ? PBS_ERR_UNSUPPORTED : cuda_status(e);
+}
+
 pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out, pbs_shape s,
                          pbs_stream_t st) {
   Dims dm;

@@ -326,8 +326,10 @@ cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const voi
     const char *fi = getenv("PBS_FAULT_INJECT");
     const int fault = (fi && strcmp(fi, "timeout") == 0) ? 1 : 0;
     if (!force_tc1 || gather) {
+      OutSet one{};
+      one.p[0] = out, one.n = 1, one.hq_total = dm.hq, one.head_offset = 0;
       const cudaError_t e =
-          launch_attn_tc2(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+          launch_attn_tc2(dm, q, kp, vp, kpos, qpos, idx, cnt, one, lse, sigma, err, fault,
                           scatter, gather, st);
       if (e != cudaErrorInvalidConfiguration) return e;
     }

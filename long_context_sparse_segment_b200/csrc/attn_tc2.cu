@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ kpos,
                     const int32_t *__restrict__ qpos, const int32_t *__restrict__ blk_idx,
-                    const int32_t *__restrict__ blk_cnt, bf16 *__restrict__ out,
+                    const int32_t *__restrict__ blk_cnt, const __grid_constant__ OutSet outs,
                     float *__restrict__ lse, Dims dm, float sl2, int *err, int fault,
                     int scatter, const bf16 *__restrict__ kg, const bf16 *__restrict__ vg) {
   using C = Cfg2<D>;
@@ -599,7 +599,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false, orow_i = -1;
       }
     }
-    bf16 *orow = out + ((size_t)t.bg * dm.n + (orow_i < 0 ? 0 : orow_i)) * D;
+    // in every output buffer, at head head_offset + g of hq_total
+    const size_t orow_off =
+        ((size_t)((t.bg / dm.hq) * outs.hq_total + outs.head_offset + t.bg % dm.hq) * dm.n +
+         (orow_i < 0 ? 0 : orow_i)) * D;
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -612,15 +615,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
-        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+        for (int o = 0; o < outs.n; ++o) {
+          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<bf16 *>(outs.p[o]) + orow_off + c * 32);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+          for (int q4 = 0; q4 < 4; ++q4)
+            dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
       }
       if (lse)
         lse[(size_t)t.bg * dm.n + orow_i] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
     } else if (valid && t.count == 0 && orow_i >= 0) {
-      for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(orow)[c] = make_uint4(0, 0, 0, 0);
+      for (int o = 0; o < outs.n; ++o)
+        for (int c = 0; c < D / 8; ++c)
+          reinterpret_cast<uint4 *>(static_cast<bf16 *>(outs.p[o]) + orow_off)[c] =
+              make_uint4(0, 0, 0, 0);
       if (lse) lse[(size_t)t.bg * dm.n + orow_i] = -INFINITY;
     }
     tc_fence_before();
@@ -631,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, bool GATHER>
 cudaError_t run2(const Dims &dm, const void *q, const void *kp, const void *vp,
                  const int32_t *kpos, const int32_t *qpos, const int32_t *idx, const int32_t *cnt,
-                 void *out, float *lse, float sigma, int *err, int fault, bool scatter,
+                 const OutSet &outs, float *lse, float sigma, int *err, int fault, bool scatter,
                  cudaStream_t st) {
   if (GATHER && !kpos) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
@@ -655,7 +663,7 @@ cudaError_t run2(const Dims &dm, const void *q, const void *kp, const void *vp,
   if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   const long long total = (long long)dm.b * dm.hq * dm.nb;
   const unsigned grid = (unsigned)((total + 1) / 2);
-  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, kpos, qpos, idx, cnt, (bf16 *)out, lse, dm,
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, kpos, qpos, idx, cnt, outs, lse, dm,
                                     sigma * kLog2e, err, fault, scatter ? 1 : 0,
                                     (const bf16 *)kp, (const bf16 *)vp);
   return cudaGetLastError();
@@ -665,20 +673,29 @@ cudaError_t run2(const Dims &dm, const void *q, const void *kp, const void *vp,
 
 cudaError_t launch_attn_tc2(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
-                            const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            int fault, bool scatter, bool gather, cudaStream_t st) {
+                            const int32_t *cnt, const OutSet &outs, float *lse, float sigma,
+                            int *err, int fault, bool scatter, bool gather, cudaStream_t st) {
   if (gather) {
     if (dm.d == 64)
-      return run2<64, true>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+      return run2<64, true>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault,
                             scatter, st);
-    return run2<128, true>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+    return run2<128, true>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault,
                            scatter, st);
   }
   if (dm.d == 64)
-    return run2<64, false>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+    return run2<64, false>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault,
                            scatter, st);
-  return run2<128, false>(dm, q, kp, vp, kpos, qpos, idx, cnt, out, lse, sigma, err, fault,
+  return run2<128, false>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault,
                           scatter, st);
+}
+
+cudaError_t launch_attn_bcast(const Dims &dm, const void *q, const void *kp, const void *vp,
+                              const int32_t *kpos, const int32_t *idx, const int32_t *cnt,
+                              const OutSet &outs, float sigma, int *err, cudaStream_t st) {
+  if (!attn_tc_supported(dm)) return cudaErrorNotSupported;
+  const cudaError_t e = launch_attn_tc2(dm, q, kp, vp, kpos, nullptr, idx, cnt, outs, nullptr,
+                                        sigma, err, 0, false, false, st);
+  return e == cudaErrorInvalidConfiguration ? cudaErrorNotSupported : e;
 }
 
 }  // namespace pbs

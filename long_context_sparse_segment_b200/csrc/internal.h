@@ -67,11 +67,26 @@ cudaError_t launch_attn_tc(const Dims &dm, const void *q, const void *kp, const 
                            const int32_t *cnt, void *out, float *lse, float sigma, int *err,
                            int fault, bool scatter, cudaStream_t st);
 
+// Where the forward writes its rows: n buffers of [b, hq_total, n, d] bf16;
+// query head g of the call lands at head head_offset + g of each. One
+// buffer with hq_total = hq and offset 0 is the plain case.
+constexpr int kMaxOuts = 8;
+struct OutSet {
+  void *p[kMaxOuts];
+  int n, hq_total, head_offset;
+};
+
 // the same forward with two query tiles per CTA (tcgen05; B = 128, d in {64, 128})
 cudaError_t launch_attn_tc2(const Dims &dm, const void *q, const void *kp, const void *vp,
                             const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
-                            const int32_t *cnt, void *out, float *lse, float sigma, int *err,
-                            int fault, bool scatter, bool gather, cudaStream_t st);
+                            const int32_t *cnt, const OutSet &outs, float *lse, float sigma,
+                            int *err, int fault, bool scatter, bool gather, cudaStream_t st);
+
+// the forward writing every row into several buffers (two-tile kernel only;
+// cudaErrorNotSupported where it does not run)
+cudaError_t launch_attn_bcast(const Dims &dm, const void *q, const void *kp, const void *vp,
+                              const int32_t *kpos, const int32_t *idx, const int32_t *cnt,
+                              const OutSet &outs, float sigma, int *err, cudaStream_t st);
 
 // the same forward on the legacy warp-MMA path
 cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const void *vp,

@@ -161,6 +161,35 @@ def attn_fwd_gather(q, k, v, kpos, qpos, blk_idx, blk_cnt, block, segment, scale
     return (o, l) if lse else o
 
 
+def attn_fwd_bcast(q, k_perm, v_perm, kpos, blk_idx, blk_cnt, block, segment, outs,
+                   head_offset=0, scale=0.0):
+    """attn_fwd writing every output row into each tensor of ``outs``
+    ([b, hq_total, n, d] bf16, on this device or mapped into its address
+    space), query head g at head ``head_offset + g`` (pbs_attn_fwd_bcast)."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_perm, "k_perm", torch.bfloat16, q.device)
+    _need(v_perm, "v_perm", torch.bfloat16, q.device)
+    if kpos is not None:
+        _need(kpos, "kpos", torch.int32, q.device)
+    _need(blk_idx, "blk_idx", torch.int32, q.device)
+    _need(blk_cnt, "blk_cnt", torch.int32, q.device)
+    if not outs:
+        raise ValueError("outs: at least one output tensor")
+    b, _, n, d = q.shape
+    hq_total = outs[0].shape[1]
+    for i, o in enumerate(outs):
+        if (o.dtype != torch.bfloat16 or not o.is_contiguous() or o.dim() != 4
+                or (o.shape[0], o.shape[2], o.shape[3]) != (b, n, d) or o.shape[1] != hq_total):
+            raise ValueError(f"outs[{i}]: contiguous bf16 [b, hq_total, n, d] expected")
+    ptrs = (ctypes.c_void_p * len(outs))(*[o.data_ptr() for o in outs])
+    shp = shape_of(q, k_perm, block, segment)
+    check(lib().pbs_attn_fwd_bcast(_ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(kpos),
+                                   _ptr(blk_idx), _ptr(blk_cnt), ptrs, len(outs), hq_total,
+                                   head_offset, shp, scale, _stream(q.device)),
+          "pbs_attn_fwd_bcast")
+    return outs
+
+
 def unpermute(o_perm, qpos, hkv, block, segment, out=None):
     """o[b, g, qpos[b, g/G, p]] = o_perm[b, g, p]."""
     _need(o_perm, "o_perm", torch.bfloat16)

@@ -135,6 +135,35 @@ def test_gathering_forward_and_order_only_permute_arguments(lib):
                            None) == _lib.ERR_INVALID_ARG
 
 
+def test_broadcast_forward_arguments(lib):
+    s = shape()
+    fake = ctypes.c_void_p(1 << 20)
+    other = ctypes.c_void_p(1 << 24)
+    outs = (ctypes.c_void_p * 9)(*([1 << 26] * 9))
+    hq = s.hq
+    call = lib.pbs_attn_fwd_bcast
+    # 1..8 outputs
+    assert call(fake, fake, fake, None, fake, fake, outs, 0, hq, 0, s, 0.0, None) == \
+        _lib.ERR_INVALID_ARG
+    assert call(fake, fake, fake, None, fake, fake, outs, 9, hq, 0, s, 0.0, None) == \
+        _lib.ERR_INVALID_ARG
+    # the call's heads must fit inside the buffers' heads
+    assert call(fake, fake, fake, None, fake, fake, outs, 2, hq, 1, s, 0.0, None) == \
+        _lib.ERR_INVALID_ARG
+    assert call(fake, fake, fake, None, fake, fake, outs, 2, 2 * hq, -1, s, 0.0, None) == \
+        _lib.ERR_INVALID_ARG
+    # an output that is an input, a misaligned output
+    alias = (ctypes.c_void_p * 2)(1 << 26, 1 << 20)
+    assert call(fake, other, other, None, other, other, alias, 2, hq, 0, s, 0.0, None) == \
+        _lib.ERR_INVALID_ARG
+    odd = (ctypes.c_void_p * 1)((1 << 26) + 8)
+    assert call(fake, fake, fake, None, fake, fake, odd, 1, hq, 0, s, 0.0, None) == \
+        _lib.ERR_INVALID_ARG
+    # only the two-tile tcgen05 forward writes several buffers
+    assert call(fake, fake, fake, None, fake, fake, outs, 2, hq, 0, shape(block=64), 0.0,
+                None) == _lib.ERR_UNSUPPORTED
+
+
 def test_fused_forward_rejects_output_aliasing_an_input(lib):
     s = shape()
     fake = ctypes.c_void_p(1 << 20)

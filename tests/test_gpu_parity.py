@@ -384,3 +384,43 @@ def test_host_buffer_path_steps_of_query_heads(name, dev, monkeypatch):
         outs[step] = o.clone()
     for step, o in outs.items():
         assert torch.equal(o, outs[w.group]), f"step of {step} heads"
+
+
+@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128", "odd_items"])
+def test_broadcast_forward_writes_every_buffer(name, dev):
+    """pbs_attn_fwd_bcast writes the forward's rows into every buffer at the
+    given head offset (as each rank of a head-sharded run writes its heads
+    into its own and its peers' outputs) and nothing else; the rows are bit
+    for bit pbs_attn_fwd's."""
+    w = CASES[name]
+    _, (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    imp = pbs.score(qd, kd, B)
+    perm = pbs.permute(imp, kd, vd, B, S, hq=w.hq)
+    idx, cnt, _ = pbs.select_blocks(qd, perm["k_perm"], perm["kbar_sum"], B, S, w.mode, w.param)
+    args = (qd, perm["k_perm"], perm["v_perm"], perm["kpos"])
+    o_ref = pbs.attn_fwd(*args, None, idx, cnt, B, S)
+    b, hq, n, d = qd.shape
+    sentinel = torch.tensor(-7.0, dtype=torch.bfloat16)
+    for n_out, total, offset in ((1, hq, 0), (3, 3 * hq, hq), (2, 2 * hq + 1, hq + 1)):
+        outs = [torch.full((b, total, n, d), -7.0, dtype=torch.bfloat16, device=dev)
+                for _ in range(n_out)]
+        pbs.attn_fwd_bcast(*args, idx, cnt, B, S, outs, head_offset=offset)
+        torch.cuda.synchronize()
+        assert pbs.device_status() == 0
+        for o in outs:
+            assert torch.equal(o[:, offset:offset + hq], o_ref)
+            rest = torch.cat([o[:, :offset], o[:, offset + hq:]], dim=1)
+            assert bool((rest.cpu() == sentinel).all())
+
+
+def test_broadcast_forward_needs_the_two_tile_kernel(dev):
+    w = CASES["d128_b64"]
+    _, (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    imp = pbs.score(qd, kd, B)
+    perm = pbs.permute(imp, kd, vd, B, S, hq=w.hq)
+    idx, cnt, _ = pbs.select_blocks(qd, perm["k_perm"], perm["kbar_sum"], B, S, w.mode, w.param)
+    with pytest.raises(pbs.PbsError):
+        pbs.attn_fwd_bcast(qd, perm["k_perm"], perm["v_perm"], perm["kpos"], idx, cnt, B, S,
+                           [torch.empty_like(qd)])
