@@ -494,10 +494,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       uint32_t v[kBN];
+      // the first half of S, then the second half in flight while the first
+      // half's row max runs; the empty asm ties each half's registers to its
+      // wait so that no use is scheduled before the data has landed
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c)
+      for (int c = 0; c < 2; ++c)
         tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
       tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 64; ++c) asm volatile("" : "+r"(v[c]));
+#pragma unroll
+      for (int c = 2; c < 4; ++c)
+        tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
+      float m8[8];
+      if (!diag) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(v[e]);
+#pragma unroll
+        for (int c = 8; c < 64; c += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], __uint_as_float(v[c + e]));
+      }
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 64; c < kBN; ++c) asm volatile("" : "+r"(v[c]));
       if (diag) {
         if (kpos) {
           // the block's carried original key positions arrived with its V' tile
@@ -524,12 +544,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // row max: eight independent chains over the 128 columns (a clock64
-      // trace measured the three-input max.f32 slower here)
-      float m8[8];
+      // trace measured the three-input max.f32 slower here); off the
+      // diagonal segment the first half was taken while the second loaded
+      if (diag) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(v[e]);
+        for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(v[e]);
 #pragma unroll
-      for (int c = 8; c < kBN; c += 8)
+        for (int c = 8; c < 64; c += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], __uint_as_float(v[c + e]));
+      }
+#pragma unroll
+      for (int c = 64; c < kBN; c += 8)
 #pragma unroll
         for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], __uint_as_float(v[c + e]));
       const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
