@@ -331,7 +331,7 @@ pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out,
  * library's (the pages do not treat host buffers).
  *
  * The work is split by KV group (batch b, KV head h: query heads
- * h*G .. h*G+G-1), in two device slots of the workspace used in turn, and
+ * h*G .. h*G+G-1), in three device slots of the workspace used in turn, and
  * inside a group by query head. On `h2d`: K, V and the last query block of
  * each head (what the scoring and the permutation need), then the query
  * heads in steps. On `compute`: the group's scoring and permutation, then
@@ -353,7 +353,7 @@ pbs_status pbs_unpermute(const void *out_perm, const int32_t *qpos, void *out,
  *   k, v         host [batch, hkv, n, d] bf16
  *   mode, param  as for pbs_select_blocks
  *   ws           device workspace of pbs_workspace_bytes(s, PBS_OP_HOST_PATH)
- *                bytes (two slots of one KV group's buffers; the size depends
+ *                bytes (three slots of one KV group's buffers; the size depends
  *                on the current device's SM count through the step size)
  * Returns PBS_ERR_UNSUPPORTED when the scoring step does not support the
  * group shape (see pbs_score).

@@ -70,6 +70,10 @@ double resolve_sigma(float scale, int d) {
 // pbs_attention_host works one KV group (batch b, KV head h: its G query
 // heads) at a time, in two device slots used in turn.
 constexpr size_t kSlotAlign = 256;
+// Device slots of the host path, used in turn by consecutive KV groups: with
+// three, group i + 1 can be copied in while group i computes and group i - 1
+// is still being copied out.
+constexpr int kSlots = 3;
 size_t aup(size_t x) { return (x + kSlotAlign - 1) & ~(kSlotAlign - 1); }
 
 Dims group_dims(const Dims &dm) {
@@ -142,7 +146,7 @@ size_t carve_slot(uint8_t *base, const Dims &g, Slot *sl) {
 }
 
 size_t host_path_ws_bytes(const Dims &dm) {
-  return 2 * carve_slot(nullptr, group_dims(dm), nullptr) + kSlotAlign;
+  return kSlots * carve_slot(nullptr, group_dims(dm), nullptr) + kSlotAlign;
 }
 
 }  // namespace
@@ -366,16 +370,16 @@ pbs_status pbs_attention_host(const void *q, const void *k, const void *v, void 
   if (!score_supported(g)) return PBS_ERR_UNSUPPORTED;
   if (ws_bytes < host_path_ws_bytes(dm)) return PBS_ERR_WORKSPACE;
   uint8_t *base = (uint8_t *)(((uintptr_t)ws + kSlotAlign - 1) & ~(uintptr_t)(kSlotAlign - 1));
-  Slot slot[2];
+  Slot slot[kSlots];
   const size_t slot_bytes = carve_slot(base, g, &slot[0]);
-  carve_slot(base + slot_bytes, g, &slot[1]);
+  for (int i = 1; i < kSlots; ++i) carve_slot(base + i * slot_bytes, g, &slot[i]);
 
   cudaStream_t cs = (cudaStream_t)compute, hst = (cudaStream_t)h2d, ds = (cudaStream_t)d2h;
   // per slot: [0] K, V and the last query block of every head copied in,
   // [1 + st] the query heads of step st copied in, [1 + steps + st] step st
   // computed, [1 + 2 steps] the slot's last output copied out
   const int G = dm.G, hs = heads_per_step(g), steps = G / hs, per_slot = 2 + 2 * steps;
-  std::vector<cudaEvent_t> evs(2 * (size_t)per_slot, nullptr);
+  std::vector<cudaEvent_t> evs(kSlots * (size_t)per_slot, nullptr);
   cudaError_t e = cudaSuccess;
   for (auto &x : evs)
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
@@ -395,7 +399,7 @@ pbs_status pbs_attention_host(const void *q, const void *k, const void *v, void 
   const int groups = dm.b * dm.hkv;
   auto at = [](const void *p, size_t off) { return (const uint8_t *)p + off; };
   for (int i = 0; i < groups && e == cudaSuccess; ++i) {
-    const int sid = i & 1, bi = i / dm.hkv, h = i % dm.hkv;
+    const int sid = i % kSlots, bi = i / dm.hkv, h = i % dm.hkv;
     const Slot &sl = slot[sid];
     const size_t qoff = ((size_t)bi * dm.hq + (size_t)h * G) * hb;  // head h*G of batch bi
     const size_t koff = ((size_t)bi * dm.hkv + h) * hb;
@@ -403,7 +407,7 @@ pbs_status pbs_attention_host(const void *q, const void *k, const void *v, void 
     // in: the slot is free once group i - 2 has been copied out. First what
     // the scoring and the permutation need (K, V, the last query block of
     // each head), then the query heads one by one
-    if (i >= 2) e = cudaStreamWaitEvent(hst, ev(sid, 1 + 2 * steps), 0);
+    if (i >= kSlots) e = cudaStreamWaitEvent(hst, ev(sid, 1 + 2 * steps), 0);
     for (int gl = 0; gl < G && e == cudaSuccess; ++gl)
       e = cudaMemcpyAsync(sq + gl * hb + restb, at(q, qoff + gl * hb + restb), lastb,
                           cudaMemcpyHostToDevice, hst);
@@ -445,7 +449,7 @@ pbs_status pbs_attention_host(const void *q, const void *k, const void *v, void 
     if (e == cudaSuccess) e = cudaEventRecord(ev(sid, 1 + 2 * steps), ds);
   }
   // work queued on the copy streams is ordered before later work on `compute`
-  for (int sid = 0; sid < 2 && sid < groups && e == cudaSuccess; ++sid)
+  for (int sid = 0; sid < kSlots && sid < groups && e == cudaSuccess; ++sid)
     e = cudaStreamWaitEvent(cs, ev(sid, 1 + 2 * steps), 0);
   for (auto &x : evs) cudaEventDestroy(x);  // released once their work completes
   return cuda_status(e);
