@@ -62,6 +62,7 @@ def test_bench_line_contract(dev):
     assert d["n_gpus"] == 1 and d["steps"] == 2 and d["warmup"] >= 3
     assert d["value"] > 0 and d["ms_per_step"] > 0 and d["higher_is_better"] is True
     assert d["config"]["workload"] == "llama8k"
+    assert d["config"]["l2"].startswith("flushed")  # 100 MB of inputs fit in L2
     assert d["gpu_launches"] == 9 * 2
     r = d["roofline"]
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
