@@ -543,8 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c > lim) v[c] = 0xff800000u;
         }
       }
-      // row max: eight independent chains over the 128 columns (a clock64
-      // trace measured the three-input max.f32 slower here); off the
+      // row max: eight independent chains over the 128 columns (the
+      // three-input max.f32 measured no faster); off the
       // diagonal segment the first half was taken while the second loaded
       if (diag) {
 #pragma unroll
