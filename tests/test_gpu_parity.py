@@ -424,3 +424,41 @@ def test_broadcast_forward_needs_the_two_tile_kernel(dev):
     with pytest.raises(pbs.PbsError):
         pbs.attn_fwd_bcast(qd, perm["k_perm"], perm["v_perm"], perm["kpos"], idx, cnt, B, S,
                            [torch.empty_like(qd)])
+
+
+@pytest.mark.parametrize("mode,param", [("threshold", 1.0), ("threshold", 0.01),
+                                        ("topk_frac", 1.0), ("topk_frac", 0.01)])
+def test_selection_extremes_against_oracle(mode, param, dev):
+    """The ends of the sparsity parameter: tau = 1 keeps blocks until the
+    whole mass (every admissible block unless the last ones carry no mass in
+    fp64), f = 1 keeps k = I + 1 blocks, and tiny tau or f keep the own
+    segment alone (it is always kept and already holds more than tau, or
+    more blocks than k). Lists bit for bit against the oracle, the top-k
+    counts against their closed form, outputs within the forward's
+    tolerance."""
+    w = CASES["gqa2k"].with_(mode=mode, param=param)
+    (q, k, v), (qd, kd, vd) = inputs(w, dev)
+    B, S = w.block, w.segment
+    imp = pbs.score(qd, kd, B)
+    perm = pbs.permute(imp, kd, vd, B, S, hq=w.hq)
+    kp = perm["k_perm"]
+    idx, cnt, _ = pbs.select_blocks(qd, kp, perm["kbar_sum"], B, S, mode, param)
+    ref_idx, ref_cnt, margin = orc.select_blocks(orc.block_means(f64(q), B),
+                                                 orc.block_means(f64(kp), B), S // B, mode,
+                                                 param, None, w.group)
+    assert compare_lists(idx, cnt, ref_idx, ref_cnt, margin) <= ref_cnt.size // 20
+    c = i64(cnt)
+    spb, nb = S // B, w.nb
+    I = np.arange(nb)
+    own = np.minimum(spb, nb - (I // spb) * spb)
+    if mode == "topk_frac":  # own segment, plus k - own earlier blocks
+        k_i = np.maximum(1, np.floor(param * (I + 1))).astype(np.int64)
+        want = own + np.minimum((I // spb) * spb, np.maximum(0, k_i - own))
+        assert np.array_equal(c, np.broadcast_to(want, c.shape))
+    if param == 0.01:
+        assert np.array_equal(c, np.broadcast_to(own, c.shape))
+    o = pbs.attn_fwd(qd, kp, perm["v_perm"], perm["kpos"], None, idx, cnt, B, S)
+    ref_o = orc.attend(f64(q), f64(kp), f64(perm["v_perm"]), i64(perm["kpos"]), None, i64(idx),
+                       i64(cnt), B)
+    assert_outputs_close(f64(o), ref_o, f"{mode} {param}")
+    assert pbs.device_status() == 0
