@@ -115,6 +115,24 @@ def test_workspace_sizes_grow_with_the_problem(lib):
     assert pbs.workspace_bytes(shape(), _lib.OP_ATTN) == 0
 
 
+def test_host_path_workspace_follows_the_step_size(lib, monkeypatch):
+    """The host path keeps three slots of one KV group's buffers; only the
+    selection scratch depends on how many query heads a step covers (one
+    step's worth is reused by the group's steps)."""
+    s = shape(hq=8, hkv=2, n=2048)  # G = 4
+    sizes = {}
+    for step in (1, 2, 4):
+        monkeypatch.setenv("PBS_HOST_STEP_HEADS", str(step))
+        sizes[step] = pbs.workspace_bytes(s, _lib.OP_HOST_PATH)
+    assert sizes[1] < sizes[2] < sizes[4]
+    nb = 2048 // GOOD["block"]
+    per_head = 8 * nb * GOOD["d"] + 2 * 8 * nb * nb  # pooled sums + scores and weights
+    assert sizes[2] - sizes[1] == 3 * per_head
+    assert sizes[4] - sizes[2] == 3 * 2 * per_head
+    monkeypatch.setenv("PBS_HOST_STEP_HEADS", "3")  # not a divisor of G: ignored
+    assert pbs.workspace_bytes(s, _lib.OP_HOST_PATH) in sizes.values()
+
+
 def test_gathering_forward_and_order_only_permute_arguments(lib):
     s = shape()
     fake = ctypes.c_void_p(1 << 20)
