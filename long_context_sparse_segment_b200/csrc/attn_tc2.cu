@@ -145,19 +145,26 @@ __device__ __forceinline__ int stream_pos(int x, int j, int cA, int cB) {
   return x == 0 ? j + min(j, cB) : j + min(j + 1, cA);
 }
 
-// Carried positions of keys 64 w + lane and 64 w + 32 + lane of block J of
-// KV head bh (w = 0, 1: the two gathering warps). A position outside block
-// J's segment is reported and replaced by the key's own index.
+// Rows of a K'/V' tile that gathering warp g (of kGatherWarps) fills:
+// [gather_lo(g), gather_lo(g + 1)), at most 64, in multiples of 4.
+constexpr int kGatherWarps = 3;
+__device__ __forceinline__ constexpr int gather_lo(int g) { return g == 3 ? kBN : 44 * g; }
+
+// Carried positions of keys lo + lane and lo + 32 + lane of block J of KV
+// head bh (rows past `rows` are not read). A position outside block J's
+// segment is reported and replaced by the key's own index.
 __device__ __forceinline__ int2 carried_rows(const int32_t *__restrict__ kpos, int bh, int J,
-                                             int w, int lane, const Dims &dm, int *err) {
-  const int p0 = J * kBN + 64 * w + lane;
+                                             int lo, int rows, int lane, const Dims &dm,
+                                             int *err) {
+  const int p0 = J * kBN + lo + lane;
   const int32_t *p = kpos + (size_t)bh * dm.n + p0;
-  int2 r = make_int2(__ldg(p), __ldg(p + 32));
+  const int unused = J * kBN;  // any key of block J: inside its segment, never read
+  int2 r = make_int2(lane < rows ? __ldg(p) : unused, lane + 32 < rows ? __ldg(p + 32) : unused);
   const int seg0 = (J / dm.spb) * dm.S;
   const unsigned span = (unsigned)min(dm.S, dm.n - seg0);  // the last segment may be short
   if ((unsigned)(r.x - seg0) >= span || (unsigned)(r.y - seg0) >= span) {
     report(err, PBS_ERR_DEVICE_ASSERT);
-    r = make_int2(p0, p0 + 32);
+    r = make_int2(lane < rows ? p0 : unused, lane + 32 < rows ? p0 + 32 : unused);
   }
   return r;
 }
@@ -199,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar->q_full, 1);
     // full: the TMA's expect-tx arrival, or one cp.async arrival per
     // gathering thread
-    const int fill_count = GATHER ? 64 : 1;
+    const int fill_count = GATHER ? 32 * kGatherWarps : 1;
     for (int s = 0; s < KS; ++s) {
       mbar_init(&bar->k_full[s], fill_count);
       mbar_init(&bar->k_empty[s], 1);
@@ -393,16 +400,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     int never = 0;
     mbar_wait(&bar->mma_done, 0, &never, nullptr);
-  } else if (GATHER) {
-    // ------------------------------------------- K, V gathers (warps 2, 3)
+  }
+  if (GATHER && warp != 1) {
+    // ---------------------------------------- K, V gathers (warps 0, 2, 3)
     // The K and V tiles in the TMA producer's order, each row read from its
-    // carried position: warp 2 fills rows 0-63 of every tile, warp 3 rows
-    // 64-127. A warp instruction moves 32 16-byte chunks (whole rows, 2 of
-    // them at d = 128) into the 128-byte-swizzled layout; each thread's
-    // cp.async arrival on the tile's full barrier (64 expected) lands when
-    // its copies have. The positions of a K block are kept for the V block
-    // of the same tile that follows it.
-    const int gw = warp - 2;
+    // carried position: warp 0 (once Q is issued) fills rows 0-43 of every
+    // tile, warp 2 rows 44-87, warp 3 rows 88-127. A warp instruction moves
+    // 32 16-byte chunks (whole rows, 2 of them at d = 128) into the
+    // 128-byte-swizzled layout; each thread's cp.async arrival on the tile's
+    // full barrier (96 expected) lands when its copies have. The positions
+    // of a K block are kept for the V block of the same tile that follows it.
+    const int gw = warp == 0 ? 0 : warp - 1;
+    const int lo = gather_lo(gw), nrows = gather_lo(gw + 1) - lo;
     constexpr int CPR = D / 8;    // 16-byte chunks per row
     constexpr int RPI = 32 / CPR; // rows per warp instruction
     const int sub = lane / CPR, ch = lane % CPR;
@@ -413,10 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto fill = [&](uint8_t *tile, const bf16 *src, int bh, int2 r) {
       const bf16 *head = src + (size_t)bh * dm.n * D + ch * 8;
 #pragma unroll 4
-      for (int it = 0; it < 64 / RPI; ++it) {
-        const int rl = it * RPI + sub;  // 0-63, warp-uniform half of r
+      for (int it = 0; it < nrows / RPI; ++it) {
+        const int rl = it * RPI + sub;  // row within the warp's range; warp-uniform half of r
         const int pos = __shfl_sync(0xffffffffu, it * RPI < 32 ? r.x : r.y, rl & 31);
-        const int row = 64 * gw + rl;
+        const int row = lo + rl;
         cp_async16(tile + col + row * 128 + ((cc ^ (row & 7)) << 4), head + (size_t)pos * D);
       }
     };
@@ -425,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int J = checked_block(t, j, dm, gw == 0 && lane == 0 ? err : nullptr);
       // the positions are read before the wait for the slot: their latency
       // hides behind it
-      const int2 r = carried_rows(kpos, t.bh, J, gw, lane, dm, err);
+      const int2 r = carried_rows(kpos, t.bh, J, lo, nrows, lane, dm, err);
       if (x) rows_b = r;
       else rows_a = r;
       if (u > 0 && !mbar_wait_warp(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 12))
@@ -443,9 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         return false;
       const int J = checked_block(t, j, dm, nullptr);
       fill(sV + s * C::TILE, vg, t.bh, x ? rows_b : rows_a);
-      if (J / dm.spb == t.segI && lane < 16)  // the mask's positions, 4 per lane
-        cp_async16(sKP + s * kBN + 64 * gw + 4 * lane,
-                   kpos + (size_t)t.bh * dm.n + (size_t)J * kBN + 64 * gw + 4 * lane);
+      if (J / dm.spb == t.segI && gw == 0)  // the mask's positions, 4 per lane
+        cp_async16(sKP + s * kBN + 4 * lane,
+                   kpos + (size_t)t.bh * dm.n + (size_t)J * kBN + 4 * lane);
       cp_async_mbar_arrive(&bar->v_full[s]);
       ++vseq;
       return true;
