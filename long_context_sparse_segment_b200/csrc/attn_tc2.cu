@@ -23,11 +23,11 @@
 //                        positions (512 bytes);
 //   warp 1               tcgen05.mma issue in the order above;
 //   (both warps run their loops warp-wide and issue from one elected lane)
-//   warps 2, 3           idle, or with GATHER (pbs_attn_fwd_gather) the K
-//                        and V tiles: each row read from the natural K, V at
-//                        its carried position with cp.async, into the
-//                        layout the TMA would write (warp 0 then loads Q
-//                        only).
+//   warps 2, 3           idle, or with GATHER (pbs_attn_fwd_gather), and
+//                        warp 0 once Q is issued, the K and V tiles: each
+//                        row read from the natural K, V at its carried
+//                        position with cp.async, into the layout the TMA
+//                        would write.
 //   warps 4-7, 8-11      softmax of tile A, of tile B: one thread per query
 //                        row (TMEM lane), all 128 key columns of a block:
 //                        mask, row max, exp2 (MUFU), P to TMEM in two
@@ -170,9 +170,9 @@ __device__ __forceinline__ int2 carried_rows(const int32_t *__restrict__ kpos, i
 }
 
 // GATHER: the permutation is applied on the fly. kg and vg are the natural
-// K and V; warps 2 and 3 fetch each block's rows by their carried positions
-// with cp.async into the same swizzled tiles the TMA would write (no K', V'
-// copies); tmK and tmV are unused.
+// K and V; warps 0 (after Q), 2 and 3 fetch each block's rows by their
+// carried positions with cp.async into the same swizzled tiles the TMA
+// would write (no K', V' copies); tmK and tmV are unused.
 template <int D, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc2_kernel(const __grid_constant__ CUtensorMap tmQ,
