@@ -151,9 +151,12 @@ def select_row(a, i_blk, spb, mode, param):
     a: block scores of the admissible key blocks 0 .. (seg(I)+1)*spb - 1,
     cut at the last block (a shorter last segment has fewer blocks).
     The margin is the smallest gap that decides the result: for THRESHOLD
-    the distance of the kept mass to tau on either side of the cut and the
-    score gap at the cut; for TOPK_FRAC the score gap at the cut. It is
-    +inf where nothing is decided.
+    the distance of the kept mass to tau on either side of the cut (the mass
+    before the last block taken, also when the walk ran out of blocks before
+    reaching tau, and the mass after it) and the score gap at the cut; for
+    TOPK_FRAC the score gap at the cut. Moving tau, or any one block score,
+    by less than the margin leaves the kept set as it is. It is +inf where
+    nothing is decided.
     """
     seg = i_blk // spb
     forced = np.arange(seg * spb, len(a))
@@ -176,7 +179,9 @@ def select_row(a, i_blk, spb, mode, param):
                 before = mass
                 mass = mass + pi[order[taken]]
                 taken += 1
-            if mass >= tau:
+            if taken > 0:
+                # tau at or below the mass before the last block ends the
+                # walk one block earlier, whether or not tau was reached
                 margin = min(margin, tau - before)
         if taken < n_earlier:
             margin = min(margin, mass - tau)
@@ -194,6 +199,18 @@ def select_row(a, i_blk, spb, mode, param):
     return kept, margin
 
 
+def block_scores(q_pooled, k_pooled, scale, group):
+    """a[b, g, I, J] = sigma * qbar_{g,I} . kbar_{h,J} with h = g // group,
+    for every pair (admissibility is applied by the caller): [b, hq, nb, nb]."""
+    b, hq, nb, d = q_pooled.shape
+    sigma = resolve_scale(scale, d)
+    a = np.empty((b, hq, nb, nb))
+    for bi in range(b):
+        for g in range(hq):
+            a[bi, g] = sigma * (q_pooled[bi, g] @ k_pooled[bi, g // group].T)
+    return a
+
+
 def select_blocks(q_pooled, k_pooled, spb, mode, param, scale, group):
     """Block lists for every (batch, query head, query block).
 
@@ -203,14 +220,13 @@ def select_blocks(q_pooled, k_pooled, spb, mode, param, scale, group):
     margin [b, hq, nb] float64).
     """
     b, hq, nb, d = q_pooled.shape
-    sigma = resolve_scale(scale, d)
     idx = np.full((b, hq, nb, nb), -1, dtype=np.int32)
     cnt = np.zeros((b, hq, nb), dtype=np.int32)
     margin = np.full((b, hq, nb), math.inf)
+    a = block_scores(q_pooled, k_pooled, scale, group)
     for bi in range(b):
         for g in range(hq):
-            kb = k_pooled[bi, g // group]
-            scores = sigma * (q_pooled[bi, g] @ kb.T)          # [nb, nb]
+            scores = a[bi, g]                                   # [nb, nb]
             for i in range(nb):
                 adm = min(nb, ((i // spb) + 1) * spb)
                 kept, mg = select_row(scores[i, :adm], i, spb, mode, param)

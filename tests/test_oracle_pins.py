@@ -320,6 +320,86 @@ def test_topk_selection_brute_force(frac):
             assert set(kept.tolist()) == set(range(seg * spb, (seg + 1) * spb)) | set(best)
 
 
+def _kept(a, i, spb, mode, tau):
+    return tuple(orc.select_row(a, i, spb, mode, tau)[0].tolist())
+
+
+def _perturbations(a, tau, mode, delta):
+    """Every single move of size delta of what the decision reads: tau up or
+    down (THRESHOLD), and each admissible block score up or down."""
+    if mode == "threshold":
+        for s in (1.0, -1.0):
+            yield a, tau + s * delta
+    for j in range(len(a)):
+        for s in (1.0, -1.0):
+            b = a.copy()
+            b[j] += s * delta
+            yield b, tau
+
+
+@pytest.mark.parametrize("mode,param", [("threshold", 0.3), ("threshold", 0.6),
+                                        ("threshold", 0.9), ("threshold", 0.999),
+                                        ("threshold", 1.0), ("topk_frac", 0.25),
+                                        ("topk_frac", 0.5), ("topk_frac", 0.75)])
+def test_selection_margin_is_the_distance_to_the_next_decision(mode, param):
+    """The margin select_row reports is what the GPU comparison trusts to
+    tell decided rows from near-ties. Pinned by brute force: moving tau or any
+    one block score by 0.99 x the margin keeps the kept set, and some such
+    move by 1.01 x the margin changes it (so the margin is neither too small
+    nor too large). An infinite margin means no move changes the set. Scores
+    are spread so that every finite margin is far above the float32 rounding
+    of tau."""
+    rng = np.random.default_rng(int(param * 1000) + len(mode))
+    spb, nseg = 2, 10
+    nb = spb * nseg
+    tested = {"finite": 0, "inf": 0}
+    for trial in range(12):
+        a_all = rng.standard_normal(nb) * 1.5
+        if param == 1.0:     # blocks whose mass is below fp64 resolution at 1
+            a_all[rng.integers(0, nb, 3)] -= 45.0
+        for i in range(nb):
+            a = a_all[:(i // spb + 1) * spb]
+            kept, margin = orc.select_row(a, i, spb, mode, param)
+            kept = tuple(kept.tolist())
+            tau = float(np.float32(param))
+            if not math.isfinite(margin):
+                tested["inf"] += 1
+                for delta in (0.5, 5.0):
+                    for b, t in _perturbations(a, tau, mode, delta):
+                        assert _kept(b, i, spb, mode, t) == kept, (i, delta)
+                continue
+            if margin < 1e-5:
+                continue       # a near-tie: reported, not compared, on the GPU
+            tested["finite"] += 1
+            for b, t in _perturbations(a, tau, mode, 0.99 * margin):
+                assert _kept(b, i, spb, mode, t) == kept, (i, margin)
+            assert any(_kept(b, i, spb, mode, t) != kept
+                       for b, t in _perturbations(a, tau, mode, 1.01 * margin)), (i, margin)
+    assert tested["finite"] >= 15 and tested["inf"] >= 12, tested
+
+
+def test_selection_margin_of_an_exhausted_threshold_walk():
+    """tau = 1 and a row whose masses, added in the walk's order, stay just
+    below 1 in fp64: every earlier block is taken without reaching tau, and
+    the decision flips once tau drops to the mass before the last block, so
+    that distance is the margin (not +inf)."""
+    rng = np.random.default_rng(21)
+    for _ in range(1000):
+        a = rng.standard_normal(6)                     # query block 4, spb 2
+        pi = np.exp(a - a.max())
+        pi /= pi.sum()
+        order = np.argsort(-a[:4], kind="stable")
+        walk = pi[4:].sum() + np.cumsum(pi[order])
+        if walk[-1] < 1.0 and walk[-2] < 1.0:
+            break
+    else:
+        pytest.fail("no row whose fp64 walk stays below 1")
+    kept, margin = orc.select_row(a, 4, 2, "threshold", 1.0)
+    assert kept.tolist() == [0, 1, 2, 3, 4, 5]
+    assert margin == 1.0 - walk[-2]
+    assert _kept(a, 4, 2, "threshold", 1.0 - 1.01 * margin) != tuple(kept.tolist())
+
+
 def test_shorter_last_segment_forces_its_own_blocks():
     q, k, v = rand_qkv(16, hq=2, hkv=1, n=96, d=8)
     res = orc.pbs_attention(q, k, v, 8, 64, "topk_frac", 0.05)
