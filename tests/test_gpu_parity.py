@@ -7,8 +7,9 @@ Split of the parity bar:
   * permute: the oracle's segment order applied to the GPU's own importance
     equals the GPU kpos bit for bit; K', V' are exact gathers; the fp64 block
     sums are exact;
-  * select: the oracle fed the GPU's permuted keys gives bit-identical lists
-    (decisions with a margin below 1e-12 are reported, not compared);
+  * select: the oracle fed the GPU's permuted keys gives bit-identical lists;
+    a decision whose oracle margin is below 1e-12 (a near-tie) is counted and
+    its list checked for validity against the rule instead;
   * forward: the oracle fed the GPU's kpos and lists is within max-abs 2e-2
     and mean-abs 2e-3.
 """
@@ -20,7 +21,7 @@ import long_context_sparse_segment_b200 as pbs
 from long_context_sparse_segment_b200.workloads import WORKLOADS, Workload, make_inputs
 from oracle import pbs_oracle as orc
 from pbs_testutil import (assert_importance_close, assert_outputs_close, compare_lists, f64,
-                          i64)
+                          i64, order_differences)
 
 pytestmark = pytest.mark.gpu
 
@@ -83,10 +84,12 @@ def test_steps_against_oracle(name, dev):
 
     idx, cnt, mask = pbs.select_blocks(qd, kp, perm["kbar_sum"], B, S, w.mode, w.param,
                                        mask=True)
-    ref_idx, ref_cnt, margin = orc.select_blocks(orc.block_means(q64, B),
-                                                 orc.block_means(f64(kp), B), S // B, w.mode,
-                                                 w.param, None, w.group)
-    assert compare_lists(idx, cnt, ref_idx, ref_cnt, margin) == 0
+    qb, kb = orc.block_means(q64, B), orc.block_means(f64(kp), B)
+    ref_idx, ref_cnt, margin = orc.select_blocks(qb, kb, S // B, w.mode, w.param, None, w.group)
+    n_amb = compare_lists(idx, cnt, ref_idx, ref_cnt, margin,
+                          scores=orc.block_scores(qb, kb, None, w.group), spb=S // B,
+                          mode=w.mode, param=w.param)
+    print(f"{name}: {n_amb} near-tie selections checked for validity")
     m = i64(mask)
     for r in np.ndindex(*ref_cnt.shape):
         assert m[r].sum() == ref_cnt[r]
@@ -108,8 +111,11 @@ def test_end_to_end_against_oracle(name, permute_q, dev):
                             permute_q=permute_q, keep=True)
     ref = orc.pbs_attention(f64(q), f64(k), f64(v), w.block, w.segment, w.mode, w.param,
                             permute_q=permute_q)
-    diff = (i64(res["kpos"]) != ref["kpos"]).mean()
-    assert diff < 0.05, f"{diff:.3%} of key slots differ"
+    # the orders may differ only at slots whose two keys have oracle
+    # importances within the scoring tolerance of each other
+    n_diff = order_differences(i64(res["kpos"]), ref["kpos"], ref["imp"])
+    print(f"{name} permute_q={permute_q}: {n_diff} of {ref['kpos'].size} key slots differ "
+          f"inside near-equal importance runs")
     assert_outputs_close(f64(res["o"]), ref["o"], name)
 
 
@@ -443,10 +449,14 @@ def test_selection_extremes_against_oracle(mode, param, dev):
     perm = pbs.permute(imp, kd, vd, B, S, hq=w.hq)
     kp = perm["k_perm"]
     idx, cnt, _ = pbs.select_blocks(qd, kp, perm["kbar_sum"], B, S, mode, param)
-    ref_idx, ref_cnt, margin = orc.select_blocks(orc.block_means(f64(q), B),
-                                                 orc.block_means(f64(kp), B), S // B, mode,
-                                                 param, None, w.group)
-    assert compare_lists(idx, cnt, ref_idx, ref_cnt, margin) <= ref_cnt.size // 20
+    qb, kb = orc.block_means(f64(q), B), orc.block_means(f64(kp), B)
+    ref_idx, ref_cnt, margin = orc.select_blocks(qb, kb, S // B, mode, param, None, w.group)
+    # rows decided by a gap below 1e-12 (tau = 1 reaches the whole mass only
+    # up to rounding) are checked for validity, every other row bit for bit
+    n_amb = compare_lists(idx, cnt, ref_idx, ref_cnt, margin,
+                          scores=orc.block_scores(qb, kb, None, w.group), spb=S // B, mode=mode,
+                          param=param)
+    print(f"{mode} {param}: {n_amb} of {ref_cnt.size} rows are near-ties, checked for validity")
     c = i64(cnt)
     spb, nb = S // B, w.nb
     I = np.arange(nb)
