@@ -123,8 +123,11 @@ pbs_status pbs_score(const void *q, const void *k, float *imp, pbs_shape s,
  *
  * - Shapes whose scoring scratch (pbs_workspace_bytes(s, PBS_OP_SCORE))
  *   exceeds the array return PBS_ERR_WORKSPACE and launch nothing.
+ * - Arguments are checked first, as pbs_score checks them: an empty shape
+ *   returns PBS_OK and a bad one its error, without touching CUDA.
  * - The first call on a device (with that device current) looks up the
- *   array's device address; make it before any stream capture.
+ *   array's device address; make it before any stream capture. A failed
+ *   lookup returns PBS_ERR_CUDA and is tried again on the next call.
  * - All calls share the array and it keeps the previous call's contents
  *   (nothing in it needs to start at zero). Calls that overlap on the GPU,
  *   from several streams or threads, race on it: serialise them.

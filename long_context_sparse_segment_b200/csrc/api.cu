@@ -34,6 +34,8 @@ int *error_word() {
   return g_err_ptr[dev];
 }
 
+}  // namespace
+
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 pbs_status check_shape(const pbs_shape &s, Dims *dm) {
@@ -60,6 +62,8 @@ pbs_status check_shape(const pbs_shape &s, Dims *dm) {
 
 bool empty(const Dims &dm) { return dm.b == 0 || dm.n == 0; }
 
+namespace {
+
 pbs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PBS_OK : PBS_ERR_CUDA; }
 
 double resolve_sigma(float scale, int d) {
@@ -68,11 +72,10 @@ double resolve_sigma(float scale, int d) {
 
 // ------------------------------------------- the host-buffer path's slots
 // pbs_attention_host works one KV group (batch b, KV head h: its G query
-// heads) at a time, in two device slots used in turn.
+// heads) at a time, in device slots used in turn by consecutive groups:
+// with three, group i + 1 can be copied in while group i computes and group
+// i - 1 is still being copied out.
 constexpr size_t kSlotAlign = 256;
-// Device slots of the host path, used in turn by consecutive KV groups: with
-// three, group i + 1 can be copied in while group i computes and group i - 1
-// is still being copied out.
 constexpr int kSlots = 3;
 size_t aup(size_t x) { return (x + kSlotAlign - 1) & ~(kSlotAlign - 1); }
 

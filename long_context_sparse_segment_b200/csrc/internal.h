@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/pbs.h"
+
 namespace pbs {
 
 struct Dims {
@@ -14,6 +16,12 @@ struct Dims {
   int spb;  // S / B
   int nseg; // ceil(n / S)
 };
+
+// Argument checks shared by the entry points: the shape (PBS_OK and *dm
+// filled, or the status to return), an empty problem, 16-byte alignment.
+pbs_status check_shape(const pbs_shape &s, Dims *dm);
+bool empty(const Dims &dm);
+bool aligned16(const void *p);
 
 // pass-1/2 importance scoring
 size_t score_ws_bytes(const Dims &dm);
