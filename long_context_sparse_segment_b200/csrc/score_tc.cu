@@ -38,6 +38,8 @@
 // together bound both passes. Every mbarrier wait is bounded
 // (PBS_ERR_TIMEOUT, the CTA drains and exits).
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK, float *__restrict__ imp,
                     float2 *__restrict__ partial, const float *__restrict__ off, Dims dm,
-                    float sl2, int nsplit, int *err) {
+                    float sl2, int nsplit, int *err, int fault) {
   using C = SCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const int R = dm.G * dm.B;
@@ -120,6 +122,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   const int t0 = (int)((long long)split * ntile / nsplit);
   const int nt = (int)((long long)(split + 1) * ntile / nsplit) - t0;
   const uint32_t tcols = W == 1 ? 128 : W == 2 ? 256 : 512;
+  // fault == PASS + 1: the first K tile is never loaded (a wait nothing will
+  // satisfy), so that this pass's bounded waits run out
+  const bool skip_first = fault == PASS + 1;
 
   if (tid == 0) {
     mbar_init(&bar->q_full, 1);
@@ -174,9 +179,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         if (u > 0 && !mbar_wait_warp(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 51)) break;
         if (leader) {
           mbar_expect_tx(&bar->k_full[s], C::TILE);
-          for (int hh = 0; hh < C::H; ++hh)
-            tma_load_2d(sK + (size_t)s * C::TILE + hh * C::HALF, &tmK, &bar->k_full[s], hh * 64,
-                        bh * dm.n + (t0 + it) * kKT);
+          if (!(skip_first && it == 0))
+            for (int hh = 0; hh < C::H; ++hh)
+              tma_load_2d(sK + (size_t)s * C::TILE + hh * C::HALF, &tmK, &bar->k_full[s],
+                          hh * 64, bh * dm.n + (t0 + it) * kKT);
         }
         __syncwarp();
         issued = it + 1;
@@ -186,7 +192,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     int never = 0;
     if (q_issued) mbar_wait(&bar->q_full, 0, &never, nullptr);
     for (int t = issued > C::KS ? issued - C::KS : 0; t < issued; ++t)
-      mbar_wait(&bar->k_full[t % C::KS], (t / C::KS) & 1, &never, nullptr);
+      if (!(skip_first && t == 0))
+        mbar_wait(&bar->k_full[t % C::KS], (t / C::KS) & 1, &never, nullptr);
   } else if (warp == pw + 1) {
     // -------------------------------------------------------- MMA issue
     // warp-wide loop (uniform waits and descriptor arithmetic), one elected
@@ -382,9 +389,21 @@ int tc_splits(const Dims &dm) {
   return s < 1 ? 1 : s;
 }
 
+// PBS_FAULT_INJECT=score_pass1 (or score_pass2) makes that pass skip the
+// first K tile of every CTA, so that its bounded waits run out and it
+// reports PBS_ERR_TIMEOUT (used by the failure-detection tests).
+int score_fault() {
+  const char *fi = getenv("PBS_FAULT_INJECT");
+  if (!fi) return 0;
+  if (strcmp(fi, "score_pass1") == 0) return 1;
+  if (strcmp(fi, "score_pass2") == 0) return 2;
+  return 0;
+}
+
 template <int D>
 cudaError_t run_tc(const Dims &dm, const void *q, const void *k, float *imp, float sigma,
                    void *ws, int *err, cudaStream_t st) {
+  const int fault = score_fault();
   const int R = dm.G * dm.B;
   const int nsplit = tc_splits(dm);
   const int bh = dm.b * dm.hkv;
@@ -405,11 +424,11 @@ cudaError_t run_tc(const Dims &dm, const void *q, const void *k, float *imp, flo
   const int threads = R + 64;
   const float sl2 = sigma * kLog2e;
   score_tc_kernel<D, 0><<<grid, threads, smem, st>>>(mq, mk, imp, partial, off, dm, sl2, nsplit,
-                                                     err);
+                                                     err, fault);
   const int total = bh * R;
   score_tc_combine<<<(total + 255) / 256, 256, 0, st>>>(partial, off, R, nsplit, total);
   score_tc_kernel<D, 1><<<grid, threads, smem, st>>>(mq, mk, imp, partial, off, dm, sl2, nsplit,
-                                                     err);
+                                                     err, fault);
   return cudaGetLastError();
 }
 

@@ -22,6 +22,16 @@ def _stream(device=None):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _call(name, *args):
+    """One C-ABI call, inside an NVTX range of its name (seen by Nsight
+    Systems beside the kernels it launches); raises on a non-OK status."""
+    torch.cuda.nvtx.range_push(name)
+    try:
+        return check(getattr(lib(), name)(*args), name)
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
 def _need(t, name, dtype, device=None):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -59,8 +69,8 @@ def score(q, k, block, segment=None, scale=0.0, ws=None, out=None):
     b, hkv, n, _ = k.shape
     imp = out if out is not None else torch.empty(b, hkv, n, dtype=torch.float32, device=q.device)
     ws, need = _workspace(shp, _lib.OP_SCORE, q.device, ws)
-    check(lib().pbs_score(_ptr(q), _ptr(k), _ptr(imp), shp, scale, _ptr(ws), need,
-                          _stream(q.device)), "pbs_score")
+    _call("pbs_score", _ptr(q), _ptr(k), _ptr(imp), shp, scale, _ptr(ws), need,
+          _stream(q.device))
     return imp
 
 
@@ -84,9 +94,9 @@ def permute(imp, k, v, block, segment, q=None, kbar=True, hq=None, materialize=T
                      if kbar else None),
         "q_perm": torch.empty_like(q) if q is not None else None,
     }
-    check(lib().pbs_permute(_ptr(imp), _ptr(k), _ptr(v), _ptr(q), _ptr(out["k_perm"]),
-                            _ptr(out["v_perm"]), _ptr(out["q_perm"]), _ptr(out["kpos"]),
-                            _ptr(out["kbar_sum"]), shp, _stream(k.device)), "pbs_permute")
+    _call("pbs_permute", _ptr(imp), _ptr(k), _ptr(v), _ptr(q), _ptr(out["k_perm"]),
+          _ptr(out["v_perm"]), _ptr(out["q_perm"]), _ptr(out["kpos"]),
+          _ptr(out["kbar_sum"]), shp, _stream(k.device))
     return out
 
 
@@ -108,9 +118,9 @@ def select_blocks(q, k_perm, kbar_sum, block, segment, mode, param=0.0, scale=0.
     cnt = cnt if cnt is not None else torch.empty(b, hq, nb, dtype=torch.int32, device=q.device)
     msk = torch.empty(b, hq, nb, nb, dtype=torch.uint8, device=q.device) if mask else None
     ws, need = _workspace(shp, _lib.OP_SELECT, q.device, ws)
-    check(lib().pbs_select_blocks(_ptr(q), _ptr(k_perm), _ptr(kbar_sum), shp, mode_id, param,
-                                  scale, _ptr(idx), _ptr(cnt), _ptr(msk), _ptr(ws), need,
-                                  _stream(q.device)), "pbs_select_blocks")
+    _call("pbs_select_blocks", _ptr(q), _ptr(k_perm), _ptr(kbar_sum), shp, mode_id, param,
+          scale, _ptr(idx), _ptr(cnt), _ptr(msk), _ptr(ws), need,
+          _stream(q.device))
     return idx, cnt, msk
 
 
@@ -131,10 +141,9 @@ def attn_fwd(q, k_perm, v_perm, kpos, qpos, blk_idx, blk_cnt, block, segment, sc
     shp = shape_of(q, k_perm, block, segment)
     o = out if out is not None else torch.empty_like(q)
     l = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if lse else None
-    fn = lib().pbs_attn_fwd_unpermute if unpermute else lib().pbs_attn_fwd
-    check(fn(_ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(kpos), _ptr(qpos), _ptr(blk_idx),
-             _ptr(blk_cnt), _ptr(o), _ptr(l), shp, scale, _stream(q.device)),
-          "pbs_attn_fwd_unpermute" if unpermute else "pbs_attn_fwd")
+    _call("pbs_attn_fwd_unpermute" if unpermute else "pbs_attn_fwd", _ptr(q), _ptr(k_perm),
+          _ptr(v_perm), _ptr(kpos), _ptr(qpos), _ptr(blk_idx), _ptr(blk_cnt), _ptr(o), _ptr(l),
+          shp, scale, _stream(q.device))
     return (o, l) if lse else o
 
 
@@ -154,10 +163,9 @@ def attn_fwd_gather(q, k, v, kpos, qpos, blk_idx, blk_cnt, block, segment, scale
     shp = shape_of(q, k, block, segment)
     o = out if out is not None else torch.empty_like(q)
     l = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if lse else None
-    check(lib().pbs_attn_fwd_gather(_ptr(q), _ptr(k), _ptr(v), _ptr(kpos), _ptr(qpos),
-                                    _ptr(blk_idx), _ptr(blk_cnt), _ptr(o), _ptr(l), shp, scale,
-                                    1 if unpermute else 0, _stream(q.device)),
-          "pbs_attn_fwd_gather")
+    _call("pbs_attn_fwd_gather", _ptr(q), _ptr(k), _ptr(v), _ptr(kpos), _ptr(qpos),
+          _ptr(blk_idx), _ptr(blk_cnt), _ptr(o), _ptr(l), shp, scale,
+          1 if unpermute else 0, _stream(q.device))
     return (o, l) if lse else o
 
 
@@ -183,10 +191,9 @@ def attn_fwd_bcast(q, k_perm, v_perm, kpos, blk_idx, blk_cnt, block, segment, ou
             raise ValueError(f"outs[{i}]: contiguous bf16 [b, hq_total, n, d] expected")
     ptrs = (ctypes.c_void_p * len(outs))(*[o.data_ptr() for o in outs])
     shp = shape_of(q, k_perm, block, segment)
-    check(lib().pbs_attn_fwd_bcast(_ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(kpos),
-                                   _ptr(blk_idx), _ptr(blk_cnt), ptrs, len(outs), hq_total,
-                                   head_offset, shp, scale, _stream(q.device)),
-          "pbs_attn_fwd_bcast")
+    _call("pbs_attn_fwd_bcast", _ptr(q), _ptr(k_perm), _ptr(v_perm), _ptr(kpos),
+          _ptr(blk_idx), _ptr(blk_cnt), ptrs, len(outs), hq_total,
+          head_offset, shp, scale, _stream(q.device))
     return outs
 
 
@@ -198,8 +205,7 @@ def unpermute(o_perm, qpos, hkv, block, segment, out=None):
     b, hq, n, d = o_perm.shape
     shp = Shape(b, hq, hkv, n, d, block, segment)
     o = out if out is not None else torch.empty_like(o_perm)
-    check(lib().pbs_unpermute(_ptr(o_perm), _ptr(qpos), _ptr(o), shp, _stream(o_perm.device)),
-          "pbs_unpermute")
+    _call("pbs_unpermute", _ptr(o_perm), _ptr(qpos), _ptr(o), shp, _stream(o_perm.device))
     return o
 
 
@@ -207,8 +213,7 @@ def device_status(device=None, detail=False):
     """Synchronise, read and clear the device error word: the pbs status code
     (0 = no kernel reported a problem), plus the diagnostic detail if asked."""
     code, where = ctypes.c_int(0), ctypes.c_int(0)
-    check(lib().pbs_get_device_status(_stream(device), ctypes.byref(code), ctypes.byref(where)),
-          "pbs_get_device_status")
+    _call("pbs_get_device_status", _stream(device), ctypes.byref(code), ctypes.byref(where))
     return (code.value, where.value) if detail else code.value
 
 
@@ -276,8 +281,8 @@ def attention_host(q, k, v, block, segment, mode="threshold", param=0.9, scale=0
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
     h2d, d2h = _copy_streams(device)
     mode_id = _lib.SEL[mode] if isinstance(mode, str) else int(mode)
-    check(lib().pbs_attention_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), shp, mode_id, param, scale,
-                                   _ptr(ws), need, _stream(device),
-                                   ctypes.c_void_p(h2d.cuda_stream),
-                                   ctypes.c_void_p(d2h.cuda_stream)), "pbs_attention_host")
+    _call("pbs_attention_host", _ptr(q), _ptr(k), _ptr(v), _ptr(o), shp, mode_id, param, scale,
+          _ptr(ws), need, _stream(device),
+          ctypes.c_void_p(h2d.cuda_stream),
+          ctypes.c_void_p(d2h.cuda_stream))
     return o

@@ -1,10 +1,12 @@
 """Failure detection without a GPU fault.
 
-The tcgen05 forward bounds every wait. PBS_FAULT_INJECT=timeout makes its K'
-loader skip the first tile load (a wait that nothing will satisfy): the
-kernel must give up after its limit (about a second), record
-PBS_ERR_TIMEOUT in the device error word, free its tensor memory and return,
-leaving the context usable. The problem is one CTA so the test takes ~1 s.
+The tcgen05 kernels bound every wait. PBS_FAULT_INJECT=timeout makes the
+forward's K' loader skip the first tile load (a wait that nothing will
+satisfy), and PBS_FAULT_INJECT=score_pass1 / score_pass2 do the same to the
+first K tile of a scoring pass: the kernel must give up after its limit
+(about a second), record PBS_ERR_TIMEOUT in the device error word, free its
+tensor memory and return, leaving the context usable. The problems are
+small, so each test takes about a second.
 """
 import pytest
 import torch
@@ -31,5 +33,31 @@ def test_bounded_wait_reports_timeout_and_context_survives(monkeypatch):
     assert code == TIMEOUT
     assert where in (32, 41), where      # MMA issuer on K', or softmax on S
     again = pbs.attn_fwd(q, k, v, None, None, idx, cnt, 128, 128)
+    assert pbs.device_status() == 0
+    assert torch.equal(again, good)
+
+
+@pytest.mark.parametrize("which,sites", [("score_pass1", (51, 53, 55)),
+                                         ("score_pass2", (51, 53, 55))])
+def test_scoring_wait_reports_timeout_and_context_survives(which, sites, monkeypatch):
+    """The same for each pass of the tcgen05 scoring: PBS_FAULT_INJECT skips
+    the pass's first K tile in every CTA; the pass gives up after its limit,
+    reports PBS_ERR_TIMEOUT and the wait that ran out, and the next call
+    gives the importance of a clean run bit for bit."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(1)
+    q = torch.randn(1, 4, 1024, 128, generator=g, device=dev).bfloat16()
+    k = torch.randn(1, 1, 1024, 128, generator=g, device=dev).bfloat16()
+    good = pbs.score(q, k, 128, 512)
+    assert pbs.device_status() == 0
+    monkeypatch.setenv("PBS_FAULT_INJECT", which)
+    pbs.score(q, k, 128, 512)
+    code, where = pbs.device_status(detail=True)
+    monkeypatch.delenv("PBS_FAULT_INJECT")
+    assert code == TIMEOUT
+    assert where in sites, where   # K loader, MMA issuer on the K tile, or a row group
+    again = pbs.score(q, k, 128, 512)
     assert pbs.device_status() == 0
     assert torch.equal(again, good)
