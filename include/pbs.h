@@ -302,7 +302,8 @@ pbs_status pbs_attn_fwd_gather(const void *q_or_qperm, const void *k,
  *   head_offset     first head this call writes, >= 0
  * The caller orders the readers after the call on every device that writes
  * into a buffer (e.g. a collective barrier on the same stream).
- * PBS_ERR_UNSUPPORTED unless B = 128 (the two-tile tcgen05 forward).
+ * Runs on the two-tile tcgen05 forwards (B = 128, and B = 64 with query
+ * tiles of two 64-row blocks); PBS_ERR_UNSUPPORTED where neither launches.
  */
 pbs_status pbs_attn_fwd_bcast(const void *q, const void *k_perm,
                               const void *v_perm, const int32_t *kpos,

@@ -18,7 +18,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpbs.so")
 
 SOURCES = ["api.cu", "score.cu", "score_static.cu", "permute.cu", "select.cu", "attn_mma.cu", "attn_tc.cu",
-           "score_tc.cu", "tmap.cu", "attn_tc2.cu",
+           "score_tc.cu", "tmap.cu", "attn_tc2.cu", "attn_tc64.cu",
            "mass_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",

@@ -331,7 +331,7 @@ pbs_status pbs_attn_fwd_bcast(const void *q, const void *k_perm, const void *v_p
     set.p[i] = outs[i];
   }
   set.n = n_out, set.hq_total = hq_total, set.head_offset = head_offset;
-  if (!attn_tc_supported(dm)) return PBS_ERR_UNSUPPORTED;
+  if (!attn_tc_supported(dm) && !attn_tc64_supported(dm)) return PBS_ERR_UNSUPPORTED;
   const float sigma = (float)resolve_sigma(scale, dm.d);
   const cudaError_t e = launch_attn_bcast(dm, q, k_perm, v_perm, kpos, blk_idx, blk_cnt, set,
                                           sigma, error_word(), (cudaStream_t)st);

@@ -303,13 +303,15 @@ cudaError_t launch_attn_mma(const Dims &dm, const void *q, const void *kp, const
 
 namespace pbs {
 
-// The tensor-core (tcgen05) kernels serve B = 128 with d = 64 or 128: by
+// The tensor-core (tcgen05) kernels serve d = 64 or 128: for B = 128 by
 // default the one with two query tiles per CTA, PBS_FORWARD=tc1 the one with
-// one tile per CTA; the warp-MMA kernel serves B = 64, and every shape under
-// PBS_FORWARD=mma (diagnostic switches for comparing the kernels). The
-// two-tile kernel refuses to launch (cudaErrorInvalidConfiguration) unless
-// it was compiled at the register count its register split assumes; the
-// one-tile kernel then runs instead.
+// one tile per CTA; for B = 64 the two-tile kernel whose tiles pair two
+// query blocks (attn_tc64.cu). The warp-MMA kernel serves every shape under
+// PBS_FORWARD=mma (diagnostic switches for comparing the kernels) and B = 64
+// with `gather`. A two-tile kernel refuses to launch
+// (cudaErrorInvalidConfiguration) unless it was compiled at the register
+// count its register split assumes; the one-tile kernel (B = 128) or the
+// warp-MMA kernel (B = 64) then runs instead.
 // PBS_FAULT_INJECT=timeout makes the tcgen05 kernels skip their first K'
 // load, so that their bounded waits run out and they report
 // PBS_ERR_TIMEOUT (used by the failure-detection test). With `gather` (keys
@@ -322,9 +324,16 @@ cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const voi
   const char *fwd = getenv("PBS_FORWARD");
   const bool force_mma = fwd && strcmp(fwd, "mma") == 0;
   const bool force_tc1 = fwd && strcmp(fwd, "tc1") == 0;
+  const char *fi = getenv("PBS_FAULT_INJECT");
+  const int fault = (fi && strcmp(fi, "timeout") == 0) ? 1 : 0;
+  if (attn_tc64_supported(dm) && !force_mma && !gather) {
+    OutSet one{};
+    one.p[0] = out, one.n = 1, one.hq_total = dm.hq, one.head_offset = 0;
+    const cudaError_t e = launch_attn_tc64(dm, q, kp, vp, kpos, qpos, idx, cnt, one, lse, sigma,
+                                           err, fault, scatter, st);
+    if (e != cudaErrorInvalidConfiguration) return e;
+  }
   if (attn_tc_supported(dm) && !force_mma) {
-    const char *fi = getenv("PBS_FAULT_INJECT");
-    const int fault = (fi && strcmp(fi, "timeout") == 0) ? 1 : 0;
     if (!force_tc1 || gather) {
       OutSet one{};
       one.p[0] = out, one.n = 1, one.hq_total = dm.hq, one.head_offset = 0;

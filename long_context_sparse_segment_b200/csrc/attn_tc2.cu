@@ -727,9 +727,13 @@ cudaError_t launch_attn_tc2(const Dims &dm, const void *q, const void *kp, const
 cudaError_t launch_attn_bcast(const Dims &dm, const void *q, const void *kp, const void *vp,
                               const int32_t *kpos, const int32_t *idx, const int32_t *cnt,
                               const OutSet &outs, float sigma, int *err, cudaStream_t st) {
-  if (!attn_tc_supported(dm)) return cudaErrorNotSupported;
-  const cudaError_t e = launch_attn_tc2(dm, q, kp, vp, kpos, nullptr, idx, cnt, outs, nullptr,
-                                        sigma, err, 0, false, false, st);
+  cudaError_t e = cudaErrorNotSupported;
+  if (attn_tc_supported(dm))
+    e = launch_attn_tc2(dm, q, kp, vp, kpos, nullptr, idx, cnt, outs, nullptr, sigma, err, 0,
+                        false, false, st);
+  else if (attn_tc64_supported(dm))
+    e = launch_attn_tc64(dm, q, kp, vp, kpos, nullptr, idx, cnt, outs, nullptr, sigma, err, 0,
+                         false, st);
   return e == cudaErrorInvalidConfiguration ? cudaErrorNotSupported : e;
 }
 

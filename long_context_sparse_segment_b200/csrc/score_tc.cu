@@ -63,7 +63,7 @@ struct SCfg {
   static constexpr uint32_t HALF = 128u * 128;    // bytes of one 64-column box
   static constexpr int KS = D == 128 ? 2 : 4;     // K ring depth
   static size_t smem(int R) {
-    return 1024 + (size_t)(R / 128) * TILE + (size_t)KS * TILE + sizeof(uint64_t) * 32 +
+    return 1024 + (size_t)((R + 127) / 128) * TILE + (size_t)KS * TILE + sizeof(uint64_t) * 32 +
            (size_t)R * 4 + 2 * kMaxW * 128 * 4 + 16;
   }
 };
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   using C = SCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const int R = dm.G * dm.B;
-  const int W = R / 128;
+  const int W = (R + 127) / 128;  // 128-row slices; the last may be half padding
   uint8_t *base = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t *sQ = base;
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         prefetch_map(&tmK);
         // probe row r = gl * B + i is row n - B + i of query head h G + gl;
         // 128-row tile r / 128 of the Q array, each tile stored as H boxes.
-        mbar_expect_tx(&bar->q_full, (uint32_t)W * C::TILE);
+        mbar_expect_tx(&bar->q_full, (uint32_t)R * D * 2);
         for (int gl = 0; gl < dm.G; ++gl) {
           const int r0 = gl * dm.B;
           const int grow = (b * dm.hq + h * dm.G + gl) * dm.n + dm.n - dm.B;
@@ -308,7 +308,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           l += s.x + s.y;
         } else {
           // ---- key key0 + lrow over probe rows 128 w + 64 hf .. + 63
+          // (rows past R pad the last slice: never loaded, never summed)
           const int rb = w * 128 + hf * 64;
+          if (rb >= R) continue;
           if (edge) {
             // probe row q (position n - B + q mod B) sees the key only if
             // q mod B >= key - (n - B); keys past n are seen by none
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         }
       }
     }
-    if (PASS == 0 && ok && nt > 0)
+    if (PASS == 0 && ok && nt > 0 && r < R)
       partial[((size_t)bh * nsplit + split) * R + r] = make_float2(m, l);
   }
   tc_fence_before();
@@ -421,7 +423,7 @@ cudaError_t run_tc(const Dims &dm, const void *q, const void *k, float *imp, flo
   float2 *partial = reinterpret_cast<float2 *>(ws);
   float *off = reinterpret_cast<float *>(partial + (size_t)bh * nsplit * R);
   const dim3 grid(nsplit, bh);
-  const int threads = R + 64;
+  const int threads = (R + 127) / 128 * 128 + 64;
   const float sl2 = sigma * kLog2e;
   score_tc_kernel<D, 0><<<grid, threads, smem, st>>>(mq, mk, imp, partial, off, dm, sl2, nsplit,
                                                      err, fault);
@@ -446,7 +448,7 @@ int sm_count() {
 
 bool score_tc_supported(const Dims &dm) {
   const int R = dm.G * dm.B;
-  if (R % 128 != 0 || R > 128 * kMaxW || (dm.B != 64 && dm.B != 128)) return false;
+  if (R % 64 != 0 || R > 128 * kMaxW || (dm.B != 64 && dm.B != 128)) return false;
   if (dm.d == 64) return SCfg<64>::smem(R) <= 227 * 1024;
   if (dm.d == 128) return SCfg<128>::smem(R) <= 227 * 1024;
   return false;

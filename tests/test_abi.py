@@ -177,9 +177,6 @@ def test_broadcast_forward_arguments(lib):
     odd = (ctypes.c_void_p * 1)((1 << 26) + 8)
     assert call(fake, fake, fake, None, fake, fake, odd, 1, hq, 0, s, 0.0, None) == \
         _lib.ERR_INVALID_ARG
-    # only the two-tile tcgen05 forward writes several buffers
-    assert call(fake, fake, fake, None, fake, fake, outs, 2, hq, 0, shape(block=64), 0.0,
-                None) == _lib.ERR_UNSUPPORTED
 
 
 def test_fused_forward_rejects_output_aliasing_an_input(lib):

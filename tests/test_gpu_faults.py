@@ -17,22 +17,25 @@ pytestmark = pytest.mark.gpu
 TIMEOUT = 4
 
 
-def test_bounded_wait_reports_timeout_and_context_survives(monkeypatch):
+@pytest.mark.parametrize("block", [128, 64])
+def test_bounded_wait_reports_timeout_and_context_survives(block, monkeypatch):
+    """The forward for B = 128 and the one for B = 64 (query tiles of two
+    64-row blocks)."""
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev).manual_seed(0)
     q, k, v = (torch.randn(1, 1, 128, 128, generator=g, device=dev).bfloat16() for _ in range(3))
-    idx, cnt, _ = pbs.select_blocks(q, k, None, 128, 128, "all")
-    good = pbs.attn_fwd(q, k, v, None, None, idx, cnt, 128, 128)
+    idx, cnt, _ = pbs.select_blocks(q, k, None, block, 128, "all")
+    good = pbs.attn_fwd(q, k, v, None, None, idx, cnt, block, 128)
     assert pbs.device_status() == 0
     monkeypatch.setenv("PBS_FAULT_INJECT", "timeout")
-    pbs.attn_fwd(q, k, v, None, None, idx, cnt, 128, 128)
+    pbs.attn_fwd(q, k, v, None, None, idx, cnt, block, 128)
     code, where = pbs.device_status(detail=True)
     monkeypatch.delenv("PBS_FAULT_INJECT")
     assert code == TIMEOUT
     assert where in (32, 41), where      # MMA issuer on K', or softmax on S
-    again = pbs.attn_fwd(q, k, v, None, None, idx, cnt, 128, 128)
+    again = pbs.attn_fwd(q, k, v, None, None, idx, cnt, block, 128)
     assert pbs.device_status() == 0
     assert torch.equal(again, good)
 

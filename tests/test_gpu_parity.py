@@ -47,6 +47,10 @@ CASES = {
     # S = N: one segment, every block forced
     "s_eq_n": Workload("s_eq_n", 1, 2, 1, 1024, 64, 64, 1024, "threshold", 0.5,
                        "uniform", 0.05),
+    # B = 64 with an odd number of query blocks and S = B (each query block of
+    # a paired tile in its own segment), GQA with G = 3
+    "b64_odd": Workload("b64_odd", 1, 3, 1, 1216, 128, 64, 64, "topk_frac", 0.3,
+                        "uniform", 0.05),
 }
 
 
@@ -207,10 +211,13 @@ def test_device_status_is_clean(dev):
     assert pbs.device_status() == 0
 
 
-@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128", "odd_items"])
+@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128", "odd_items", "tiny", "d128_b64",
+                                  "s_eq_n", "b64_odd"])
 def test_tensor_core_and_warp_mma_forwards_agree(name, dev, monkeypatch):
     """The tcgen05 forward and the warp-MMA forward on the same lists, each
-    against the oracle."""
+    against the oracle. B = 64 shapes run the kernel whose 128-row tiles pair
+    two query blocks (with an odd number of query blocks in b64_odd, the last
+    tile's second block lies past the end)."""
     w = CASES[name]
     (q, k, v), (qd, kd, vd) = inputs(w, dev)
     B, S = w.block, w.segment
@@ -231,8 +238,9 @@ def test_tensor_core_and_warp_mma_forwards_agree(name, dev, monkeypatch):
 
 
 SCORE_SHAPES = {
-    # (batch, hq, hkv, n, d, B): G*B = 512, 256, 384 and 128 take the tcgen05
-    # kernel, G*B = 64 the warp-MMA kernel
+    # (batch, hq, hkv, n, d, B): every G*B up to 512 takes the tcgen05 kernel;
+    # where G*B is not a multiple of 128 (64, 192) the last 128-row slice of
+    # probe rows is half padding
     "r512_d128": (1, 8, 2, 2048, 128, 128),
     "r256_b2": (2, 4, 2, 1280, 128, 128),
     "r384": (1, 6, 2, 1536, 128, 128),
@@ -240,6 +248,8 @@ SCORE_SHAPES = {
     # B = 64 probe rows, n % 128 == 64: the last key tile is half past the end
     "r128_b64_tail": (1, 4, 2, 1088, 128, 64),
     "r64_mma": (1, 4, 4, 1024, 128, 64),
+    "r64_d64": (1, 1, 1, 1024, 64, 64),
+    "r192_b64": (2, 6, 2, 1088, 128, 64),
 }
 
 
@@ -392,7 +402,7 @@ def test_host_buffer_path_steps_of_query_heads(name, dev, monkeypatch):
         assert torch.equal(o, outs[w.group]), f"step of {step} heads"
 
 
-@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128", "odd_items"])
+@pytest.mark.parametrize("name", ["gqa2k", "ragged", "d64_b128", "odd_items", "d128_b64", "tiny"])
 def test_broadcast_forward_writes_every_buffer(name, dev):
     """pbs_attn_fwd_bcast writes the forward's rows into every buffer at the
     given head offset (as each rank of a head-sharded run writes its heads
@@ -418,18 +428,6 @@ def test_broadcast_forward_writes_every_buffer(name, dev):
             assert torch.equal(o[:, offset:offset + hq], o_ref)
             rest = torch.cat([o[:, :offset], o[:, offset + hq:]], dim=1)
             assert bool((rest.cpu() == sentinel).all())
-
-
-def test_broadcast_forward_needs_the_two_tile_kernel(dev):
-    w = CASES["d128_b64"]
-    _, (qd, kd, vd) = inputs(w, dev)
-    B, S = w.block, w.segment
-    imp = pbs.score(qd, kd, B)
-    perm = pbs.permute(imp, kd, vd, B, S, hq=w.hq)
-    idx, cnt, _ = pbs.select_blocks(qd, perm["k_perm"], perm["kbar_sum"], B, S, w.mode, w.param)
-    with pytest.raises(pbs.PbsError):
-        pbs.attn_fwd_bcast(qd, perm["k_perm"], perm["v_perm"], perm["kpos"], idx, cnt, B, S,
-                           [torch.empty_like(qd)])
 
 
 @pytest.mark.parametrize("mode,param", [("threshold", 1.0), ("threshold", 0.01),
