@@ -65,9 +65,19 @@ def parse():
     ap.add_argument("--gather-kv", action="store_true",
                     help="the forward reads K, V through the key order (pbs_attn_fwd_gather); "
                          "the permutation writes only the order and block sums")
+    ap.add_argument("--block", type=int, choices=[64, 128], default=None,
+                    help="the workload with another block size B (the method's free "
+                         "parameter; its segment size and selection unchanged)")
     ap.add_argument("--profile", action="store_true",
                     help="time the steps only (no dense, end-to-end or CPU legs), for ncu")
     return ap.parse_args()
+
+
+def workload_of(args):
+    w = WORKLOADS[args.config]
+    if args.block and args.block != w.block:
+        w = w.with_(name=f"{w.name}_b{args.block}", block=args.block)
+    return w
 
 
 def peaks():
@@ -314,7 +324,7 @@ def gpu_arm(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    w = WORKLOADS[args.config]
+    w = workload_of(args)
     sharded = args.shard == "heads" and world > 1
     w_full = w
     if sharded:
@@ -573,7 +583,7 @@ def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    w = WORKLOADS[args.config]
+    w = workload_of(args)
     whole = oracle_fits_whole(w)
     if whole:   # the whole workload, drawn on the host with the same recipe
         q, k, v, _ = make_inputs(w)
