@@ -409,7 +409,13 @@ def gpu_arm(args):
     attn_launch_ms = per["attn"] / len(layers)
     value, ms, _ = job_throughput(flops_per_step, ms, dist, dev)
     pk, pk_kind = peaks()
-    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    # the burst GEMM figure for a forward timed in steps of well under a
+    # second; the sustained one (a seconds-long loop under the power cap) for
+    # steps of a second or more, such as the 32-layer stack
+    long_step = ms >= 1000.0
+    peak_burst = pk.get("bf16_tflops", pk.get("bf16_tflops_sustained"))
+    peak_sust = pk.get("bf16_tflops_sustained", peak_burst)
+    peak = peak_sust if long_step else peak_burst
     attn_tflops = flops_per_step / len(layers) / (attn_launch_ms * 1e-3) / 1e12
 
     if args.profile:
@@ -452,7 +458,8 @@ def gpu_arm(args):
         "roofline": {"kernel": "pbs_attn_fwd", "bound": "tensor",
                      "achieved": round(attn_tflops, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peak, 4), "peak_kind":
-                     f"{pk_kind} bf16 dense, sustained",
+                     f"{pk_kind} bf16 dense, {'sustained' if long_step else 'burst'}",
+                     "frac_of_sustained": round(attn_tflops / peak_sust, 4),
                      "traffic": None if args.gather_kv else traffic_for(w)},
     }
     if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.profile):
