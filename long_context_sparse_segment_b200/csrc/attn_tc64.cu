@@ -10,23 +10,27 @@
 //
 // The MMA's M is 128 rows, so a query tile is two consecutive 64-row query
 // blocks 2P and 2P + 1 of one head, each with its own list of kept key
-// blocks. The tile walks the union of the two lists (merged, ascending): per
-// key block J one 128 x 64 product S = Q K'_J^T and one O += P V'_J with
-// K = 64; the rows of a query block whose list does not hold J see the
-// whole block masked, so each row attends to exactly its own list. A CTA
-// takes two such tiles, A and B, and the tensor core alternates between
-// them as in the B = 128 kernel (attn_tc2.cu):
-//   S_A(0), S_B(0), then per block j:  O_A += P_A(j) V'_A(j), S_A(j+1),
-//                                      O_B += P_B(j) V'_B(j), S_B(j+1).
-// TMEM: S_x in columns 128 x .. 128 x + 63 (P is written over its first 32
-// columns as bf16 pairs), O_x in 256 + 128 x. 384 threads:
-//   warp 0        TMA: Q_A, Q_B, then 64-row K' and V' tiles in the order
-//                 the tensor core consumes them; a V' tile of a block in the
-//                 own segment of either query block brings the block's
-//                 carried key positions;
+// blocks. The tile walks the union of the two lists (merged, ascending),
+// two key blocks at a time: a step j takes union entries 2j and 2j + 1
+// (J0, J1), loads them as the two 64-row halves of one 128-row K' tile and
+// V' tile (two TMA boxes each), and runs one 128 x 128 product
+// S = Q [K'_J0; K'_J1]^T and one O += P [V'_J0; V'_J1] with K = 128. The
+// rows of a query block whose list does not hold J0 (J1) see that half of
+// the step masked, so each row attends to exactly its own list; an odd last
+// entry is loaded twice and its second copy masked everywhere. A CTA takes
+// two such tiles, A and B, and the tensor core alternates between them as in
+// the B = 128 kernel (attn_tc2.cu):
+//   S_A(0), S_B(0), then per step j:  O_A += P_A(j) V'_A(j), S_A(j+1),
+//                                     O_B += P_B(j) V'_B(j), S_B(j+1).
+// TMEM: S_A, S_B (P over the first 64 columns of its S as bf16 pairs), O_A,
+// O_B. 384 threads:
+//   warp 0        TMA: Q_A, Q_B, then K' and V' tiles in the order the
+//                 tensor core consumes them; a key block in the own segment
+//                 of either query block brings its carried key positions
+//                 with its V' half;
 //   warp 1        tcgen05.mma issue;
 //   warps 4-11    softmax of tile A, of tile B: one thread per query row,
-//                 the 64 key columns of a block in registers.
+//                 the 128 key columns of a step in registers.
 // Each role walks the same merged list. Every mbarrier wait is bounded; on
 // expiry the CTA records PBS_ERR_TIMEOUT, drains what it issued, frees TMEM
 // and exits.
@@ -44,7 +48,8 @@ using namespace tc;
 
 constexpr int kBM = 128;  // query rows per tile (MMA M): two query blocks
 constexpr int kQB = 64;   // rows per query block
-constexpr int kBN = 64;   // keys per block
+constexpr int kSB = 64;   // keys per block
+constexpr int kBN = 128;  // keys per step: two blocks
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;   // per thread at launch (checked on the host)
 constexpr int kCtrlRegs = 56;      // warps 0-3 after setmaxnreg.dec
@@ -55,13 +60,12 @@ constexpr float kRescaleLog2 = 8.0f;  // move the running max only past 2^8
 
 template <int D>
 struct Cfg64 {
-  static constexpr int H = D / 64;                             // 128-byte atoms per row
-  static constexpr uint32_t QTILE = (uint32_t)kBM * D * 2;     // bytes of a query tile
-  static constexpr uint32_t QHALF = (uint32_t)kBM * 128;       // one 64-column box of it
-  static constexpr uint32_t KTILE = (uint32_t)kBN * D * 2;     // bytes of a K' or V' tile
-  static constexpr uint32_t KHALF = (uint32_t)kBN * 128;       // one 64-column box of it
-  static constexpr int KS = 4;                                 // K' ring depth
-  static constexpr int VS = 4;                                 // V' ring depth
+  static constexpr int H = D / 64;                           // 128-byte atoms per row
+  static constexpr uint32_t TILE = (uint32_t)kBM * D * 2;    // bytes of a 128-row tile
+  static constexpr uint32_t HALF = (uint32_t)kBM * 128;      // one 64-column box of it
+  static constexpr uint32_t SUB = (uint32_t)kSB * 128;       // its 64-row part (one TMA box)
+  static constexpr int KS = D == 128 ? 2 : 4;                // K' ring depth
+  static constexpr int VS = D == 128 ? 3 : 4;                // V' ring depth
 };
 
 template <int D>
@@ -72,8 +76,7 @@ struct Bars64 {
 
 template <int D>
 constexpr size_t smem64() {
-  return 1024 + 2 * (size_t)Cfg64<D>::QTILE +
-         (size_t)(Cfg64<D>::KS + Cfg64<D>::VS) * Cfg64<D>::KTILE +
+  return 1024 + 2 * (size_t)Cfg64<D>::TILE + (size_t)(Cfg64<D>::KS + Cfg64<D>::VS) * Cfg64<D>::TILE +
          (size_t)Cfg64<D>::VS * kBN * 4 + sizeof(Bars64<D>) + 16;
 }
 static_assert(smem64<128>() <= 232448, "shared memory (d = 128)");
@@ -129,6 +132,17 @@ struct Union {
     for (int h = 0; h < 2; ++h) l[h] = t.list[h], c[h] = t.c[h], i[h] = 0;
   }
   __device__ __forceinline__ bool more() const { return i[0] < c[0] || i[1] < c[1]; }
+  // the next step's two blocks (the second a masked copy of the first when
+  // the union has one entry left) and which lists hold each
+  __device__ __forceinline__ void next2(int nb, int *err, int (&J)[2], int (&in)[2]) {
+    J[0] = next(nb, err, &in[0]);
+    if (more()) {
+      J[1] = next(nb, err, &in[1]);
+    } else {
+      J[1] = J[0];
+      in[1] = 0;
+    }
+  }
   // the next block and which of the two lists hold it (bit h)
   __device__ __forceinline__ int next(int nb, int *err, int *in) {
     int v[2];
@@ -150,7 +164,7 @@ struct Union {
   }
 };
 
-// Position of block j of tile x (0 = A, 1 = B) in the interleaved stream
+// Position of step j of tile x (0 = A, 1 = B) in the interleaved stream
 // A0 B0 A1 B1 ... (a list that has ended drops out).
 __device__ __forceinline__ int stream_pos(int x, int j, int cA, int cB) {
   return x == 0 ? j + min(j, cB) : j + min(j + 1, cA);
@@ -170,14 +184,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t *sQ = base;                          // [2] query tiles
-  uint8_t *sK = sQ + 2 * C::QTILE;             // [KS] K' tiles
-  uint8_t *sV = sK + KS * C::KTILE;            // [VS] V' tiles
-  int32_t *sKP = reinterpret_cast<int32_t *>(sV + VS * C::KTILE);  // [VS][kBN]
+  uint8_t *sQ = base;                    // [2] query tiles
+  uint8_t *sK = sQ + 2 * C::TILE;        // [KS] K' tiles of two blocks
+  uint8_t *sV = sK + KS * C::TILE;       // [VS] V' tiles of two blocks
+  int32_t *sKP = reinterpret_cast<int32_t *>(sV + VS * C::TILE);  // [VS][kBN]
   Bars64<D> *bar = reinterpret_cast<Bars64<D> *>(sKP + VS * kBN);
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
-  int *s_cnt = const_cast<int *>(s_abort) + 1;  // [2] union lengths
+  int *s_cnt = const_cast<int *>(s_abort) + 1;  // [2] steps of each tile
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int total = dm.b * dm.hq * ((dm.nb + 1) / 2);
@@ -197,18 +211,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bar->s_full[x], 1);
       mbar_init(&bar->p_full[x][0], 4);  // the four warps of the tile's softmax,
-      mbar_init(&bar->p_full[x][1], 4);  // for keys 0-31 and 32-63 of P
+      mbar_init(&bar->p_full[x][1], 4);  // for the step's first and second block
       mbar_init(&bar->o_final[x], 1);
     }
     mbar_init(&bar->mma_done, 1);
     *s_abort = 0;
-    // every role walks the same unions; their lengths are counted once here
+    // every role walks the same unions; their step counts are found once here
     for (int x = 0; x < 2; ++x) {
       Union u;
       u.init(x ? tB : tA);
       int n = 0, in;
       while (u.more()) u.next(dm.nb, err, &in), ++n;
-      s_cnt[x] = n;
+      s_cnt[x] = (n + 1) / 2;
     }
     fence_barrier_init();
   }
@@ -227,9 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
   if (warp == 0) {
     // ------------------------------------------------------- TMA loads
-    // Order: K'_A(0), K'_B(0), then per block j and tile x: V'_x(j),
-    // K'_x(j+1) -- the tensor core's order. The whole warp runs the loop;
-    // one elected lane issues the copies.
+    // Order: K'_A(0), K'_B(0), then per step j and tile x: V'_x(j),
+    // K'_x(j+1) -- the tensor core's order. A tile is two 64-row boxes per
+    // 64 columns, one from each of the step's blocks. The whole warp runs
+    // the loop; one elected lane issues the copies.
     const bool leader = elect_one();
     bool q_issued = false;
     int kseq = 0, vseq = 0;
@@ -238,31 +253,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_map(&tmK);
       prefetch_map(&tmV);
       if (leader) {
-        mbar_expect_tx(&bar->q_full, ((cA > 0) + (cB > 0)) * C::QTILE);
+        mbar_expect_tx(&bar->q_full, ((cA > 0) + (cB > 0)) * C::TILE);
         for (int x = 0; x < 2; ++x) {
           const Tile64 &t = x ? tB : tA;
           if ((x ? cB : cA) == 0) continue;
           for (int h = 0; h < C::H; ++h)
-            tma_load_2d(sQ + x * C::QTILE + h * C::QHALF, &tmQ, &bar->q_full, h * 64,
+            tma_load_2d(sQ + x * C::TILE + h * C::HALF, &tmQ, &bar->q_full, h * 64,
                         t.bg * dm.n + t.P * kBM);
         }
       }
       __syncwarp();
       q_issued = true;
-      Union uk[2], uv[2];
-      uk[0].init(tA), uk[1].init(tB), uv[0].init(tA), uv[1].init(tB);
+      // a step's K' tile is loaded before its V' tile, so the pair of
+      // blocks found for the K' tile is kept for the V' tile that follows
+      Union uA, uB;
+      uA.init(tA), uB.init(tB);
+      int JA[2] = {0, 0}, JB[2] = {0, 0};
       auto load_k = [&](int x) -> bool {
         const int s = kseq % KS, u = kseq / KS;
         if (u > 0 && !mbar_wait_warp(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 11))
           return false;
-        int in;
-        const int J = uk[x].next(dm.nb, nullptr, &in);
+        int in[2];
+        int(&J)[2] = x ? JB : JA;
+        (x ? uB : uA).next2(dm.nb, nullptr, J, in);
+        const int row0 = (x ? tB : tA).bh * dm.n;
         if (leader) {
-          mbar_expect_tx(&bar->k_full[s], C::KTILE);
+          mbar_expect_tx(&bar->k_full[s], C::TILE);
           if (!(fault == 1 && kseq == 0))
             for (int h = 0; h < C::H; ++h)
-              tma_load_2d(sK + s * C::KTILE + h * C::KHALF, &tmK, &bar->k_full[s], h * 64,
-                          (x ? tB : tA).bh * dm.n + J * kBN);
+              for (int b = 0; b < 2; ++b)
+                tma_load_2d(sK + s * C::TILE + h * C::HALF + b * C::SUB, &tmK, &bar->k_full[s],
+                            h * 64, row0 + J[b] * kSB);
         }
         __syncwarp();
         ++kseq;
@@ -273,18 +294,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u > 0 && !mbar_wait_warp(&bar->v_empty[s], (u - 1) & 1, s_abort, err, 21))
           return false;
         const Tile64 &t = x ? tB : tA;
-        int in;
-        const int J = uv[x].next(dm.nb, nullptr, &in);
-        const int sj = J / dm.spb;
-        const bool with_pos = kpos && ((t.has[0] && sj == t.seg[0]) || (t.has[1] && sj == t.seg[1]));
+        const int(&J)[2] = x ? JB : JA;
+        bool with_pos[2];
+        for (int b = 0; b < 2; ++b) {
+          const int sj = J[b] / dm.spb;
+          with_pos[b] = kpos && ((t.has[0] && sj == t.seg[0]) || (t.has[1] && sj == t.seg[1]));
+        }
         if (leader) {
-          mbar_expect_tx(&bar->v_full[s], C::KTILE + (with_pos ? kBN * 4 : 0));
+          mbar_expect_tx(&bar->v_full[s], C::TILE + (with_pos[0] + with_pos[1]) * kSB * 4);
           for (int h = 0; h < C::H; ++h)
-            tma_load_2d(sV + s * C::KTILE + h * C::KHALF, &tmV, &bar->v_full[s], h * 64,
-                        t.bh * dm.n + J * kBN);
-          if (with_pos)
-            bulk_load(sKP + s * kBN, kpos + (size_t)t.bh * dm.n + (size_t)J * kBN, kBN * 4,
-                      &bar->v_full[s]);
+            for (int b = 0; b < 2; ++b)
+              tma_load_2d(sV + s * C::TILE + h * C::HALF + b * C::SUB, &tmV, &bar->v_full[s],
+                          h * 64, t.bh * dm.n + J[b] * kSB);
+          for (int b = 0; b < 2; ++b)
+            if (with_pos[b])
+              bulk_load(sKP + s * kBN + b * kSB, kpos + (size_t)t.bh * dm.n + (size_t)J[b] * kSB,
+                        kSB * 4, &bar->v_full[s]);
         }
         __syncwarp();
         ++vseq;
@@ -317,21 +342,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t hi = sw128_desc_hi(1024);
     const uint32_t lo_q = sw128_desc_lo(smem_u32(sQ), 16);
     const uint32_t lo_k = sw128_desc_lo(smem_u32(sK), 16);
-    const uint32_t lo_v = sw128_desc_lo(smem_u32(sV), C::KHALF);
+    const uint32_t lo_v = sw128_desc_lo(smem_u32(sV), C::HALF);
     int ks = 0, kph = 0, vs = 0, vph = 0;
     bool ok = cmax > 0 && mbar_wait_warp(&bar->q_full, 0, s_abort, err, 31);
     if (ok) tc_fence_after();
-    // S_x = Q_x K'^T: A = Q_x (128 rows), B = the 64-row K' tile, K-major
+    // S_x = Q_x K'^T: A = Q_x, B = the step's K' tile, both K-major
     auto qk = [&](int x) -> bool {
       if (!mbar_wait_warp(&bar->k_full[ks], kph, s_abort, err, 32)) return false;
       tc_fence_after();
-      const uint32_t lq = lo_q + x * (C::QTILE >> 4), lk = lo_k + ks * (C::KTILE >> 4);
+      const uint32_t lq = lo_q + x * (C::TILE >> 4), lk = lo_k + ks * (C::TILE >> 4);
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t sa = ((kk >> 2) * C::QHALF + (kk & 3) * 32) >> 4;
-          const uint32_t sb = ((kk >> 2) * C::KHALF + (kk & 3) * 32) >> 4;
-          mma_ss(tbase + x * 128, desc_words(lq + sa, hi), desc_words(lk + sb, hi), kIdQK,
+          const uint32_t step = ((kk >> 2) * C::HALF + (kk & 3) * 32) >> 4;
+          mma_ss(tbase + x * 128, desc_words(lq + step, hi), desc_words(lk + step, hi), kIdQK,
                  kk > 0);
         }
         mma_commit(&bar->k_empty[ks]);
@@ -341,14 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (++ks == KS) ks = 0, kph ^= 1;
       return true;
     };
-    // O_x += P_x V': A = P_x from TMEM (bf16 pairs over S_x), B = the V' tile
-    // (MN-major); 16 keys per MMA, the first half of P while the softmax
-    // still writes the second; the first block of a tile overwrites O_x
+    // O_x += P_x V': A = P_x from TMEM (bf16 pairs over S_x), B = the V'
+    // tile (MN-major); the first block's 64 keys while the softmax still
+    // writes the second's; the first step of a tile overwrites O_x
     auto pv = [&](int x, int j) -> bool {
       if (!mbar_wait_warp(&bar->p_full[x][0], j & 1, s_abort, err, 33)) return false;
       if (!mbar_wait_warp(&bar->v_full[vs], vph, s_abort, err, 34)) return false;
       tc_fence_after();
-      const uint32_t lv = lo_v + vs * (C::KTILE >> 4);
+      const uint32_t lv = lo_v + vs * (C::TILE >> 4);
       for (int h = 0; h < 2; ++h) {
         if (h == 1) {
           if (!mbar_wait_warp(&bar->p_full[x][1], j & 1, s_abort, err, 35)) return false;
@@ -418,10 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     Union un;
     un.init(t);
     for (int j = 0; j < cnt && ok; ++j) {
-      int in;
-      const int J = un.next(dm.nb, nullptr, &in);
-      const bool mine = real && ((in >> hr) & 1);  // this row's list keeps J
-      const bool diag = J / dm.spb == t.seg[hr];
+      int J[2], in[2];
+      un.next2(dm.nb, nullptr, J, in);
       if (!mbar_wait_warp(&bar->s_full[x], j & 1, s_abort, err, 41)) {
         ok = false;
         break;
@@ -429,41 +451,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t v[kBN];
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+      for (int c = 0; c < kBN / 32; ++c)
         tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < kBN; ++c) asm volatile("" : "+r"(v[c]));
-      if (!mine) {
-        // a block only the other query block keeps, or no query here
+      // per block of the step: masked whole where this row's list does not
+      // keep it (or the row has no query), per element in the own segment
+      const bool mine0 = real && (in[0] >> hr & 1), mine1 = real && (in[1] >> hr & 1);
+      const bool diag0 = mine0 && J[0] / dm.spb == t.seg[hr];
+      const bool diag1 = mine1 && J[1] / dm.spb == t.seg[hr];
+      const int4 *kp4 = nullptr;
+      if (kpos && __any_sync(0xffffffffu, diag0 || diag1)) {
+        // the blocks' carried original key positions arrived with the V' tile
+        const int seq = stream_pos(x, j, cA, cB);
+        const int vsl = seq % VS;
+        if (!mbar_wait_warp(&bar->v_full[vsl], (seq / VS) & 1, s_abort, err, 42)) {
+          ok = false;
+          break;
+        }
+        kp4 = reinterpret_cast<const int4 *>(sKP + vsl * kBN);
+      }
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) v[c] = 0xff800000u;  // -inf
-      } else if (diag) {
-        if (kpos) {
-          // the block's carried original key positions arrived with its V' tile
-          const int seq = stream_pos(x, j, cA, cB);
-          const int vsl = seq % VS;
-          if (!mbar_wait_warp(&bar->v_full[vsl], (seq / VS) & 1, s_abort, err, 42)) {
-            ok = false;
-            break;
+      for (int b = 0; b < 2; ++b) {
+        const bool mine = b ? mine1 : mine0, diag = b ? diag1 : diag0;
+        if (!mine) {
+#pragma unroll
+          for (int c = 0; c < kSB; ++c) v[b * kSB + c] = 0xff800000u;  // -inf
+        } else if (diag && kp4) {
+#pragma unroll
+          for (int c4 = 0; c4 < kSB / 4; ++c4) {
+            const int4 p = kp4[b * (kSB / 4) + c4];
+            const int c = b * kSB + 4 * c4;
+            if (p.x > qp) v[c] = 0xff800000u;
+            if (p.y > qp) v[c + 1] = 0xff800000u;
+            if (p.z > qp) v[c + 2] = 0xff800000u;
+            if (p.w > qp) v[c + 3] = 0xff800000u;
           }
-          const int4 *kp4 = reinterpret_cast<const int4 *>(sKP + vsl * kBN);
+        } else if (diag) {
+          const int lim = qp - J[b] * kSB;  // last visible column of the block
 #pragma unroll
-          for (int c4 = 0; c4 < kBN / 4; ++c4) {
-            const int4 p = kp4[c4];
-            if (p.x > qp) v[4 * c4] = 0xff800000u;
-            if (p.y > qp) v[4 * c4 + 1] = 0xff800000u;
-            if (p.z > qp) v[4 * c4 + 2] = 0xff800000u;
-            if (p.w > qp) v[4 * c4 + 3] = 0xff800000u;
-          }
-        } else {
-          const int lim = qp - J * kBN;  // last visible column
-#pragma unroll
-          for (int c = 0; c < kBN; ++c)
-            if (c > lim) v[c] = 0xff800000u;
+          for (int c = 0; c < kSB; ++c)
+            if (c > lim) v[b * kSB + c] = 0xff800000u;
         }
       }
-      // row max: eight independent chains over the 64 columns
+      // row max: eight independent chains over the 128 columns
       float m8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(v[e]);
@@ -481,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float mu = m_used == -INFINITY ? 0.f : m_used;
       __syncwarp();  // reconverge after the per-row branches before aligned TMEM work
-      // O_x already holds every block before j; rows with alpha == 1
+      // O_x already holds every step before j; rows with alpha == 1
       // multiply by one when any row of the warp rescales
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
@@ -496,8 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       // p = 2^(s sigma log2(e) - m) on the hardware exp2; P to TMEM as bf16
-      // pairs over the first 32 columns of S_x, each half (keys 0-31, 32-63)
-      // signalled as soon as it is written
+      // pairs over the first 64 columns of S_x, each block's half signalled
+      // as soon as it is written
       const float2 neg_m2 = make_float2(-mu, -mu);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
@@ -514,9 +546,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[e] = pack_bf16(p.x, p.y);
         }
         tmem_st16(tS + c * 16, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        warp_arrive(&bar->p_full[x][c], lane);
+        if (c == 1 || c == 3) {
+          tmem_wait_st();
+          tc_fence_before();
+          warp_arrive(&bar->p_full[x][c >> 1], lane);
+        }
       }
       const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
       l = l * alpha + (a.x + a.y);
@@ -575,8 +609,8 @@ cudaError_t run64(const Dims &dm, const void *q, const void *kp, const void *vp,
                   cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_tile_map(&mq, q, (uint64_t)dm.b * dm.hq * dm.n, D, kBM) ||
-      !make_tile_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D, kBN) ||
-      !make_tile_map(&mv, vp, (uint64_t)dm.b * dm.hkv * dm.n, D, kBN))
+      !make_tile_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D, kSB) ||
+      !make_tile_map(&mv, vp, (uint64_t)dm.b * dm.hkv * dm.n, D, kSB))
     return cudaErrorInvalidValue;
   constexpr size_t smem = smem64<D>();
   auto kern = attn_tc64_kernel<D>;
