@@ -307,8 +307,8 @@ namespace pbs {
 // default the one with two query tiles per CTA, PBS_FORWARD=tc1 the one with
 // one tile per CTA; for B = 64 the two-tile kernel whose tiles pair two
 // query blocks (attn_tc64.cu). The warp-MMA kernel serves every shape under
-// PBS_FORWARD=mma (diagnostic switches for comparing the kernels) and B = 64
-// with `gather`. A two-tile kernel refuses to launch
+// PBS_FORWARD=mma (diagnostic switches for comparing the kernels). A
+// two-tile kernel refuses to launch
 // (cudaErrorInvalidConfiguration) unless it was compiled at the register
 // count its register split assumes; the one-tile kernel (B = 128) or the
 // warp-MMA kernel (B = 64) then runs instead.
@@ -326,11 +326,11 @@ cudaError_t launch_attn(const Dims &dm, const void *q, const void *kp, const voi
   const bool force_tc1 = fwd && strcmp(fwd, "tc1") == 0;
   const char *fi = getenv("PBS_FAULT_INJECT");
   const int fault = (fi && strcmp(fi, "timeout") == 0) ? 1 : 0;
-  if (attn_tc64_supported(dm) && !force_mma && !gather) {
+  if (attn_tc64_supported(dm) && !force_mma) {
     OutSet one{};
     one.p[0] = out, one.n = 1, one.hq_total = dm.hq, one.head_offset = 0;
     const cudaError_t e = launch_attn_tc64(dm, q, kp, vp, kpos, qpos, idx, cnt, one, lse, sigma,
-                                           err, fault, scatter, st);
+                                           err, fault, scatter, gather, st);
     if (e != cudaErrorInvalidConfiguration) return e;
   }
   if (attn_tc_supported(dm) && !force_mma) {

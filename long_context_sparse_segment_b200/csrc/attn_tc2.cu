@@ -733,7 +733,7 @@ cudaError_t launch_attn_bcast(const Dims &dm, const void *q, const void *kp, con
                         false, false, st);
   else if (attn_tc64_supported(dm))
     e = launch_attn_tc64(dm, q, kp, vp, kpos, nullptr, idx, cnt, outs, nullptr, sigma, err, 0,
-                         false, st);
+                         false, false, st);
   return e == cudaErrorInvalidConfiguration ? cudaErrorNotSupported : e;
 }
 

@@ -29,6 +29,10 @@
 //                 of either query block brings its carried key positions
 //                 with its V' half;
 //   warp 1        tcgen05.mma issue;
+//   warps 2, 3    idle, or with GATHER (pbs_attn_fwd_gather), and warp 0
+//                 once Q is issued, the K' and V' tiles: each row read from
+//                 the natural K, V at its carried position with cp.async,
+//                 into the layout the TMA would write;
 //   warps 4-11    softmax of tile A, of tile B: one thread per query row,
 //                 the 128 key columns of a step in registers.
 // Each role walks the same merged list. Every mbarrier wait is bounded; on
@@ -164,13 +168,48 @@ struct Union {
   }
 };
 
+// Rows of a step's K'/V' tile that gathering warp g (of three) fills:
+// [gather_lo(g), gather_lo(g + 1)), at most 64, in multiples of 4.
+__device__ __forceinline__ constexpr int gather_lo(int g) { return g == 3 ? kBN : 44 * g; }
+
+// Carried positions of rows lo + lane and lo + 32 + lane of a step's tile
+// (row r is key r mod 64 of block J[r / 64]) of KV head bh; rows past `rows`
+// are not read. A position outside its block's segment is reported and
+// replaced by the key's own index.
+__device__ __forceinline__ int2 carried_rows(const int32_t *__restrict__ kpos, int bh,
+                                             const int (&J)[2], int lo, int rows, int lane,
+                                             const Dims &dm, int *err) {
+  int r2[2];
+  for (int k = 0; k < 2; ++k) {
+    const int r = lo + lane + 32 * k;
+    const int Jr = J[r >> 6];
+    const int own = Jr * kSB + (r & (kSB - 1));
+    if (lane + 32 * k >= rows) {
+      r2[k] = Jr * kSB;  // any key of the block: inside its segment, never read
+      continue;
+    }
+    int pos = __ldg(kpos + (size_t)bh * dm.n + own);
+    const int seg0 = (Jr / dm.spb) * dm.S;
+    const unsigned span = (unsigned)min(dm.S, dm.n - seg0);  // the last segment may be short
+    if ((unsigned)(pos - seg0) >= span) {
+      report(err, PBS_ERR_DEVICE_ASSERT);
+      pos = own;
+    }
+    r2[k] = pos;
+  }
+  return make_int2(r2[0], r2[1]);
+}
+
 // Position of step j of tile x (0 = A, 1 = B) in the interleaved stream
 // A0 B0 A1 B1 ... (a list that has ended drops out).
 __device__ __forceinline__ int stream_pos(int x, int j, int cA, int cB) {
   return x == 0 ? j + min(j, cB) : j + min(j + 1, cA);
 }
 
-template <int D>
+// GATHER: the permutation is applied on the fly. kg and vg are the natural
+// K and V; warps 0 (after Q), 2 and 3 fetch each step's rows by their
+// carried positions with cp.async (no K', V' copies); tmK and tmV are unused.
+template <int D, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc64_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
@@ -178,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const int32_t *__restrict__ qpos, const int32_t *__restrict__ blk_idx,
                      const int32_t *__restrict__ blk_cnt, const __grid_constant__ OutSet outs,
                      float *__restrict__ lse, Dims dm, float sl2, int *err, int fault,
-                     int scatter) {
+                     int scatter, const bf16 *__restrict__ kg, const bf16 *__restrict__ vg) {
   using C = Cfg64<D>;
   constexpr int KS = C::KS, VS = C::VS;
   extern __shared__ uint8_t smem_raw[];
@@ -200,12 +239,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&bar->q_full, 1);
+    // full: the TMA's expect-tx arrival, or one cp.async arrival per
+    // gathering thread
+    const int fill_count = GATHER ? 96 : 1;
     for (int s = 0; s < KS; ++s) {
-      mbar_init(&bar->k_full[s], 1);
+      mbar_init(&bar->k_full[s], fill_count);
       mbar_init(&bar->k_empty[s], 1);
     }
     for (int s = 0; s < VS; ++s) {
-      mbar_init(&bar->v_full[s], 1);
+      mbar_init(&bar->v_full[s], fill_count);
       mbar_init(&bar->v_empty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -250,8 +292,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kseq = 0, vseq = 0;
     if (cmax > 0) {
       prefetch_map(&tmQ);
-      prefetch_map(&tmK);
-      prefetch_map(&tmV);
+      if (!GATHER) {
+        prefetch_map(&tmK);
+        prefetch_map(&tmV);
+      }
       if (leader) {
         mbar_expect_tx(&bar->q_full, ((cA > 0) + (cB > 0)) * C::TILE);
         for (int x = 0; x < 2; ++x) {
@@ -315,8 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++vseq;
         return true;
       };
-      bool ok = true;
-      if (cA > 0) ok = load_k(0);
+      bool ok = !GATHER;  // with GATHER, warps 0, 2 and 3 load K' and V' below
+      if (ok && cA > 0) ok = load_k(0);
       if (ok && cB > 0) ok = load_k(1);
       for (int j = 0; j < cmax && ok; ++j)
         for (int x = 0; x < 2 && ok; ++x) {
@@ -350,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto qk = [&](int x) -> bool {
       if (!mbar_wait_warp(&bar->k_full[ks], kph, s_abort, err, 32)) return false;
       tc_fence_after();
+      if constexpr (GATHER) fence_proxy_async_smem();  // rows written by cp.async
       const uint32_t lq = lo_q + x * (C::TILE >> 4), lk = lo_k + ks * (C::TILE >> 4);
       if (leader) {
 #pragma unroll
@@ -372,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_warp(&bar->p_full[x][0], j & 1, s_abort, err, 33)) return false;
       if (!mbar_wait_warp(&bar->v_full[vs], vph, s_abort, err, 34)) return false;
       tc_fence_after();
+      if constexpr (GATHER) fence_proxy_async_smem();
       const uint32_t lv = lo_v + vs * (C::TILE >> 4);
       for (int h = 0; h < 2; ++h) {
         if (h == 1) {
@@ -413,6 +459,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     int never = 0;
     mbar_wait(&bar->mma_done, 0, &never, nullptr);
+  }
+  if (GATHER && warp != 1) {
+    // ---------------------------------------- K, V gathers (warps 0, 2, 3)
+    // The K' and V' tiles in the TMA loader's order, each row read from its
+    // carried position: warp 0 (once Q is issued) fills rows 0-43 of every
+    // tile, warp 2 rows 44-87, warp 3 rows 88-127. A warp instruction moves
+    // 32 16-byte chunks into the 128-byte-swizzled layout; each thread's
+    // cp.async arrival on the tile's full barrier (96 expected) lands when
+    // its copies have. The positions of a step's K' tile are kept for its V'
+    // tile, which also brings the positions of the step's two blocks.
+    const int gw = warp == 0 ? 0 : warp - 1;
+    const int lo = gather_lo(gw), nrows = gather_lo(gw + 1) - lo;
+    constexpr int CPR = D / 8;    // 16-byte chunks per row
+    constexpr int RPI = 32 / CPR; // rows per warp instruction
+    const int sub = lane / CPR, ch = lane % CPR;
+    const uint32_t col = (uint32_t)(ch >> 3) * C::HALF;  // 128-byte column block
+    const int cc = ch & 7;
+    int2 rows_a = make_int2(0, 0), rows_b = rows_a;
+    int JA[2] = {0, 0}, JB[2] = {0, 0};
+    Union uA, uB;
+    uA.init(tA), uB.init(tB);
+    int kseq = 0, vseq = 0;
+    auto fill = [&](uint8_t *tile, const bf16 *src, int bh, int2 r) {
+      const bf16 *head = src + (size_t)bh * dm.n * D + ch * 8;
+#pragma unroll 4
+      for (int it = 0; it < nrows / RPI; ++it) {
+        const int rl = it * RPI + sub;  // row within the warp's range; warp-uniform half of r
+        const int pos = __shfl_sync(0xffffffffu, it * RPI < 32 ? r.x : r.y, rl & 31);
+        const int row = lo + rl;
+        cp_async16(tile + col + row * 128 + ((cc ^ (row & 7)) << 4), head + (size_t)pos * D);
+      }
+    };
+    auto load_k = [&](int x) -> bool {
+      const int s = kseq % KS, u = kseq / KS;
+      const Tile64 &t = x ? tB : tA;
+      int in[2];
+      int(&J)[2] = x ? JB : JA;
+      (x ? uB : uA).next2(dm.nb, nullptr, J, in);
+      // the positions are read before the wait for the slot: their latency
+      // hides behind it
+      const int2 r = carried_rows(kpos, t.bh, J, lo, nrows, lane, dm, err);
+      if (x) rows_b = r;
+      else rows_a = r;
+      if (u > 0 && !mbar_wait_warp(&bar->k_empty[s], (u - 1) & 1, s_abort, err, 12))
+        return false;
+      if (!(fault == 1 && kseq == 0)) {
+        fill(sK + s * C::TILE, kg, t.bh, r);
+        cp_async_mbar_arrive(&bar->k_full[s]);
+      }
+      ++kseq;
+      return true;
+    };
+    auto load_v = [&](int x) -> bool {
+      const int s = vseq % VS, u = vseq / VS;
+      if (u > 0 && !mbar_wait_warp(&bar->v_empty[s], (u - 1) & 1, s_abort, err, 22))
+        return false;
+      const Tile64 &t = x ? tB : tA;
+      const int(&J)[2] = x ? JB : JA;
+      fill(sV + s * C::TILE, vg, t.bh, x ? rows_b : rows_a);
+      if (gw == 0)  // the mask's positions of both blocks, 4 per lane
+        cp_async16(sKP + s * kBN + 4 * lane,
+                   kpos + (size_t)t.bh * dm.n + (size_t)J[lane >> 4] * kSB + 4 * (lane & 15));
+      cp_async_mbar_arrive(&bar->v_full[s]);
+      ++vseq;
+      return true;
+    };
+    bool ok = true;
+    if (cA > 0) ok = load_k(0);
+    if (ok && cB > 0) ok = load_k(1);
+    for (int j = 0; j < cmax && ok; ++j)
+      for (int x = 0; x < 2 && ok; ++x) {
+        const int c = x ? cB : cA;
+        if (j >= c) continue;
+        ok = load_v(x);
+        if (ok && j + 1 < c) ok = load_k(x);
+      }
+    cp_async_wait_all();  // every copy lands before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -602,18 +725,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool GATHER>
 cudaError_t run64(const Dims &dm, const void *q, const void *kp, const void *vp,
                   const int32_t *kpos, const int32_t *qpos, const int32_t *idx, const int32_t *cnt,
                   const OutSet &outs, float *lse, float sigma, int *err, int fault, bool scatter,
                   cudaStream_t st) {
+  if (GATHER && !kpos) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
-  if (!make_tile_map(&mq, q, (uint64_t)dm.b * dm.hq * dm.n, D, kBM) ||
-      !make_tile_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D, kSB) ||
-      !make_tile_map(&mv, vp, (uint64_t)dm.b * dm.hkv * dm.n, D, kSB))
+  if (!make_tile_map(&mq, q, (uint64_t)dm.b * dm.hq * dm.n, D, kBM)) return cudaErrorInvalidValue;
+  if (GATHER) {
+    mk = mq, mv = mq;  // unused: K and V rows are gathered with cp.async
+  } else if (!make_tile_map(&mk, kp, (uint64_t)dm.b * dm.hkv * dm.n, D, kSB) ||
+             !make_tile_map(&mv, vp, (uint64_t)dm.b * dm.hkv * dm.n, D, kSB)) {
     return cudaErrorInvalidValue;
+  }
   constexpr size_t smem = smem64<D>();
-  auto kern = attn_tc64_kernel<D>;
+  auto kern = attn_tc64_kernel<D, GATHER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -626,7 +753,8 @@ cudaError_t run64(const Dims &dm, const void *q, const void *kp, const void *vp,
   const long long total = (long long)dm.b * dm.hq * ((dm.nb + 1) / 2);
   const unsigned grid = (unsigned)((total + 1) / 2);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, kpos, qpos, idx, cnt, outs, lse, dm,
-                                    sigma * kLog2e, err, fault, scatter ? 1 : 0);
+                                    sigma * kLog2e, err, fault, scatter ? 1 : 0,
+                                    (const bf16 *)kp, (const bf16 *)vp);
   return cudaGetLastError();
 }
 
@@ -637,12 +765,19 @@ bool attn_tc64_supported(const Dims &dm) { return dm.B == 64 && (dm.d == 128 || 
 cudaError_t launch_attn_tc64(const Dims &dm, const void *q, const void *kp, const void *vp,
                              const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                              const int32_t *cnt, const OutSet &outs, float *lse, float sigma,
-                             int *err, int fault, bool scatter, cudaStream_t st) {
+                             int *err, int fault, bool scatter, bool gather, cudaStream_t st) {
+  if (gather) {
+    if (dm.d == 64)
+      return run64<64, true>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault,
+                             scatter, st);
+    return run64<128, true>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault,
+                            scatter, st);
+  }
   if (dm.d == 64)
-    return run64<64>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault, scatter,
-                     st);
-  return run64<128>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault, scatter,
-                    st);
+    return run64<64, false>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault,
+                            scatter, st);
+  return run64<128, false>(dm, q, kp, vp, kpos, qpos, idx, cnt, outs, lse, sigma, err, fault,
+                           scatter, st);
 }
 
 }  // namespace pbs

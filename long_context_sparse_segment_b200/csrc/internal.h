@@ -92,12 +92,13 @@ cudaError_t launch_attn_tc2(const Dims &dm, const void *q, const void *kp, const
 
 // the same forward for key blocks of B = 64 (tcgen05, d in {64, 128}): a
 // 128-row query tile is two 64-row query blocks walking the union of their
-// lists (no gathering mode)
+// lists, two key blocks per step; with `gather` K and V rows are read
+// through kpos as in launch_attn_tc2
 bool attn_tc64_supported(const Dims &dm);
 cudaError_t launch_attn_tc64(const Dims &dm, const void *q, const void *kp, const void *vp,
                              const int32_t *kpos, const int32_t *qpos, const int32_t *idx,
                              const int32_t *cnt, const OutSet &outs, float *lse, float sigma,
-                             int *err, int fault, bool scatter, cudaStream_t st);
+                             int *err, int fault, bool scatter, bool gather, cudaStream_t st);
 
 // the forward writing every row into several buffers (the two-tile tcgen05
 // kernels only; cudaErrorNotSupported where they do not run)

@@ -25,20 +25,23 @@ def dev():
 
 @pytest.mark.parametrize("queries", ["natural", "fused", "separate"])
 @pytest.mark.parametrize("gather_kv", [False, True])
-def test_timed_step_computes_the_path(queries, gather_kv, dev):
-    """The step bench.py times gives, in every mode, the output of the
-    path's own entry point in the matching query mode."""
+@pytest.mark.parametrize("block", [128, 64])
+def test_timed_step_computes_the_path(queries, gather_kv, block, dev):
+    """The step bench.py times gives, in every mode and for both block
+    sizes, the output of the path's own entry point in the matching query
+    and key-fetch mode."""
     sys.path.insert(0, ROOT)
     import bench
 
-    w = Workload("bench2k", 1, 8, 2, 2048, 128, 128, 512, "topk_frac", 0.3, "per_segment", 0.02)
+    w = Workload("bench2k", 1, 8, 2, 2048, 128, block, 512, "topk_frac", 0.3, "per_segment",
+                 0.02)
     layer = bench.Layer(w, dev, 0, seed_offset=0, gather_kv=gather_kv, queries=queries)
     for _ in range(2):  # the second step reuses the first one's buffers
         o, cnt = bench.run_layer(layer)
     torch.cuda.synchronize()
     assert pbs.device_status() == 0
     ref = pbs.pbs_attention(layer.q, layer.k, layer.v, w.block, w.segment, w.mode, w.param,
-                            permute_q=queries != "natural")
+                            permute_q=queries != "natural", gather_kv=gather_kv)
     assert torch.equal(o, ref)
     assert int(cnt.sum()) > 0
 
@@ -72,3 +75,13 @@ def test_bench_line_contract(dev):
     assert e["value"] > 0
     assert e["h2d_bytes_per_step"] == 2 * w.batch * (w.hq + 2 * w.hkv) * w.n * w.d
     assert e["d2h_bytes_per_step"] == 2 * w.batch * w.hq * w.n * w.d
+
+
+def test_bench_block_option(dev):
+    """--block 64 runs the workload with 64-key blocks (same segment and
+    selection) and says so in its config."""
+    d = run_bench("--config", "llama8k", "--block", "64", "--steps", "2", "--warmup", "3",
+                  "--no-cpu-baseline", "--e2e-steps", "1")
+    assert d["config"]["workload"] == "llama8k_b64" and d["config"]["block"] == 64
+    assert d["config"]["segment"] == WORKLOADS["llama8k"].segment
+    assert d["value"] > 0 and d["roofline"]["achieved"] > 0

@@ -93,6 +93,14 @@ def test_llama8k_full_size(dev):
     assert_importance_close(f64(res["imp"]), orc.score(f64(q), f64(k), B))
 
 
+def test_llama32k_block64_full_size(dev):
+    """The 32K layer with 64-key blocks (the B = 64 tcgen05 scoring and
+    forward) at full size: key orders of every head, lists and sampled
+    output blocks of three heads against the oracle."""
+    w = WORKLOADS["llama32k"].with_(name="llama32k_b64", block=64)
+    check_full_size(w, dev, heads=[0, 17, 31], blocks=sample_blocks(w.nb, w.segment // w.block))
+
+
 def test_llama32k_full_size(dev):
     w = WORKLOADS["llama32k"]
     check_full_size(w, dev, heads=[0, 13, 31], blocks=sample_blocks(w.nb, w.segment // w.block))
