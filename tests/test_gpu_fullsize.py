@@ -120,6 +120,34 @@ def test_llama128k_top25_full_size(dev):
     assert torch.equal(res["cnt"][0].long(), want.expand(w.hq, -1))
 
 
+def test_llama512k_full_size(dev):
+    """The largest context the bench runs (524,288 keys): Q and O hold 2^31
+    bf16 values (4 GiB) and the block lists 2^29 entries, so byte offsets
+    leave the 32-bit range. Orders of every head exact, gathers exact, one
+    KV head's importance, two heads' lists and sampled output blocks against
+    the oracle, the top-k counts of every row, and the last query block of
+    the last head (the last rows of O)."""
+    w = WORKLOADS["llama512k"]
+    B, S = w.block, w.segment
+    q, k, v, res = check_full_size(w, dev, heads=[0, 29], blocks=sample_blocks(w.nb, S // B))
+    I = torch.arange(w.nb, device=dev)
+    spb = S // B
+    k_i = torch.clamp((float(np.float32(w.param)) * (I + 1).double()).floor().long(), min=1)
+    own = torch.clamp(w.nb - (I // spb) * spb, max=spb)
+    earlier = (I // spb) * spb
+    want = own + torch.minimum(earlier, torch.clamp(k_i - own, min=0))
+    assert torch.equal(res["cnt"][0].long(), want.expand(w.hq, -1))
+    # the last query block of the last head: the last rows of O
+    g, hk = w.hq - 1, (w.hq - 1) // w.group
+    kp = f64(res["k_perm"][0:1, hk:hk + 1])
+    vp = f64(res["v_perm"][0:1, hk:hk + 1])
+    ref = orc.attend_blocks(f64(q[0:1, g:g + 1]), kp, vp, i64(res["kpos"][0:1, hk:hk + 1]), None,
+                            i64(res["idx"][0:1, g:g + 1]), i64(res["cnt"][0:1, g:g + 1]), B,
+                            [(0, 0, w.nb - 1)])
+    got = f64(res["o"][0, g, (w.nb - 1) * B:w.nb * B])[None]
+    assert_outputs_close(got, ref, "llama512k last block of the last head")
+
+
 def test_llama128k_all_blocks_is_dense_causal(dev):
     w = WORKLOADS["llama128k"]
     B, S = w.block, w.segment
