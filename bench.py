@@ -68,6 +68,10 @@ def parse():
     ap.add_argument("--block", type=int, choices=[64, 128], default=None,
                     help="the workload with another block size B (the method's free "
                          "parameter; its segment size and selection unchanged)")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture each layer's step as one CUDA graph after the warm-up and "
+                         "replay it in the timed region: the same kernels without the host's "
+                         "per-launch overhead, which bounds the small configs")
     ap.add_argument("--profile", action="store_true",
                     help="time the steps only (no dense, end-to-end or CPU legs), for ncu")
     return ap.parse_args()
@@ -374,8 +378,26 @@ def gpu_arm(args):
     flops_per_step = block_flops(w, total_blocks)
 
     names = ("score", "permute", "select", "attn", "unpermute", "gather")
+    graphs = None
+    if args.graph:
+        if gathering != "none":
+            raise SystemExit("--graph runs the path without --gather-output")
+        # one graph per layer, with event-record nodes around its steps
+        # (external events: replays record them, read after each step)
+        gevs = [{n: (torch.cuda.Event(enable_timing=True, external=True),
+                     torch.cuda.Event(enable_timing=True, external=True)) for n in names}
+                for _ in layers]
+        graphs = []
+        for L, ge in zip(layers, gevs):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step_layer(L, ge)
+            graphs.append(g)
+        for g in graphs:
+            g.replay()
+        torch.cuda.synchronize()
     evs = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for n in names} for _ in range(args.steps * len(layers))]
+            for n in names} for _ in range(0 if graphs else args.steps * len(layers))]
     # inputs that fit in L2 (the small configs) would stay there from one
     # step to the next: then each step is timed on its own and a 256 MB
     # write between steps, outside the timed events, flushes L2
@@ -388,24 +410,36 @@ def gpu_arm(args):
         dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(dev)
+    per_sum = {n: 0.0 for n in names}
     i = 0
     for k in range(args.steps):
         if flush is not None:
             flush.fill_(k & 0xff)
         marks[k][0].record()
-        for L in layers:
-            step_layer(L, evs[i])
-            i += 1
+        if graphs is None:
+            for L in layers:
+                step_layer(L, evs[i])
+                i += 1
+        else:
+            for g in graphs:
+                g.replay()
         marks[k][1].record()
+        if graphs is not None:  # the graphs' events hold this step's times
+            torch.cuda.synchronize()
+            for ge in gevs:
+                for n in names:
+                    per_sum[n] += ge[n][0].elapsed_time(ge[n][1])
     torch.cuda.synchronize()
     clock_info = clocks.stop()
     if dist:
         dist.barrier()
-    if flush is None:  # back to back: the whole region
+    if flush is None and graphs is None:  # back to back: the whole region
         ms = marks[0][0].elapsed_time(marks[-1][1]) / args.steps
-    else:
+    else:  # each step bracketed by its own events
         ms = sum(a.elapsed_time(b) for a, b in marks) / args.steps
-    per = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) / args.steps for n in names}
+    if graphs is None:
+        per_sum = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) for n in names}
+    per = {n: v / args.steps for n, v in per_sum.items()}
     attn_launch_ms = per["attn"] / len(layers)
     value, ms, _ = job_throughput(flops_per_step, ms, dist, dev)
     pk, pk_kind = peaks()
@@ -444,7 +478,8 @@ def gpu_arm(args):
                    "kv": "gathered inside the forward" if args.gather_kv else "permuted copies",
                    "queries": {"natural": "natural order",
                                "fused": "permuted, inverse fused into the forward",
-                               "separate": "permuted, inverse as its own step"}[args.queries]},
+                               "separate": "permuted, inverse as its own step"}[args.queries],
+                   **({"launch": "one CUDA graph per layer, replayed"} if graphs else {})},
         "density": round(total_blocks / (len(layers) * w.batch * w.hq * w.nb * (w.nb + 1) / 2), 4),
         "breakdown_ms": {n: round(v, 4) for n, v in per.items()},
         "dense_attn_ms": round(dense_ms * len(layers), 4),

@@ -46,7 +46,7 @@ constexpr int kWarps = kThreads / 32;
 
 // selection shared memory: per warp, the kept flags of its row and a digit
 // histogram
-size_t sel_smem(int nb) { return (size_t)kWarps * ((size_t)nb + 256 * 4) + 64; }
+size_t sel_smem(int nb) { return (size_t)kWarps * ((size_t)nb + 256 * 8) + 64; }
 
 __device__ __forceinline__ double f64_from_order_key(unsigned long long u) {
   return __longlong_as_double(
@@ -181,8 +181,11 @@ __global__ void __launch_bounds__(kThreads)
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const long long rowid = (long long)blockIdx.x * kWarps + w;
   if (rowid >= (long long)dm.b * dm.hq * nb) return;  // whole warp; no block barrier follows
-  unsigned *hists = reinterpret_cast<unsigned *>(smem);  // [kWarps][256]
-  unsigned char *flag = reinterpret_cast<unsigned char *>(hists + kWarps * 256) + (size_t)w * nb;
+  // per warp: a 256-bin digit histogram (32-bit counts for TOP-K, 64-bit
+  // fixed-point masses for THRESHOLD), then the row's kept flags
+  unsigned long long *hist64 = reinterpret_cast<unsigned long long *>(smem) + w * 256;
+  unsigned char *flag =
+      reinterpret_cast<unsigned char *>(smem) + (size_t)kWarps * 256 * 8 + (size_t)w * nb;
   const int bg = (int)(rowid / nb);
   const bool scored = mode == PBS_SEL_THRESHOLD || mode == PBS_SEL_TOPK_FRAC;
 
@@ -211,7 +214,7 @@ __global__ void __launch_bounds__(kThreads)
         // reaches the number still needed.
         // The bits all keys share are skipped: they would send every key to
         // one histogram bin.
-        unsigned *hist = hists + w * 256;
+        unsigned *hist = reinterpret_cast<unsigned *>(hist64);
         unsigned long long pre = 0;
         const int top = common_prefix(key, f0, lane, &pre);
         int need = t;
@@ -288,13 +291,84 @@ __global__ void __launch_bounds__(kThreads)
         if (mass_ge(0ull) < tau) {
           all_earlier = true;  // the mass never reaches tau: every block
         } else {
-          // largest value whose mass still reaches tau; it lies between the
-          // smallest and largest key, so the bits they share are fixed
+          // The cut: the largest key whose mass from the top (with the own
+          // segment's) reaches tau. Found one 8-bit digit at a time from the
+          // top, as TOP-K finds its count: among the keys that share the
+          // digits found so far, the masses per value of the next digit
+          // (fixed point in units of 2^-62, whose integer sums do not depend
+          // on their order), and the digit at which the mass from the top
+          // reaches what is still needed. The fixed point resolves the mass
+          // to ~1e-17; should it not reach what the fp64 sums above say is
+          // there, the cut is found bit by bit on the fp64 sums instead.
           unsigned long long k = 0;
           const int top = common_prefix(key, f0, lane, &k);
-          for (int bit = top; bit >= 0; --bit) {
-            const unsigned long long cand = k | (1ull << bit);
-            if (mass_ge(cand) >= tau) k = cand;
+          bool found = top < 0;  // all keys equal: the common key
+          if (!found) {
+            constexpr double kFx = 4611686018427387904.0;  // 2^62
+            const unsigned long long tau_fx = __double2ull_rn(tau * kFx);
+            const unsigned long long own_fx = __double2ull_rn(own * kFx);
+            unsigned long long need = tau_fx > own_fx ? tau_fx - own_fx : 1ull;
+            const int first = (top / 8) * 8;  // the byte holding the top bit
+            unsigned long long pmask = first + 8 >= 64 ? 0ull : ~((1ull << (first + 8)) - 1);
+            unsigned long long pre = k & pmask;
+            found = true;
+            for (int shift = first; shift >= 0 && found; shift -= 8) {
+              for (int d = lane; d < 256; d += 32) hist64[d] = 0ull;
+              __syncwarp();
+              for (int J = lane; J < f0; J += 32) {
+                const unsigned long long kj = key[J];
+                if ((kj & pmask) == pre)
+                  atomicAdd(&hist64[(unsigned)(kj >> shift) & 255u], __double2ull_rn(pi[J] * kFx));
+              }
+              __syncwarp();
+              // lane l holds digits 255 - 8l .. 248 - 8l (descending)
+              unsigned long long c[8], tot = 0;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) tot += (c[e] = hist64[255 - 8 * lane - e]);
+              unsigned long long incl = tot;  // inclusive prefix over lanes
+#pragma unroll
+              for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
+              }
+              const unsigned long long excl = incl - tot;
+              const unsigned hit = __ballot_sync(0xffffffffu, excl < need && incl >= need);
+              if (hit == 0u) {
+                found = false;
+                break;
+              }
+              const int src = __ffs(hit) - 1;
+              int digit = 0;
+              unsigned long long above = 0;
+              if (lane == src) {
+                unsigned long long run = excl;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  if (run + c[e] >= need) {
+                    digit = 255 - 8 * lane - e;
+                    break;
+                  }
+                  run += c[e];
+                }
+                above = run;
+              }
+              digit = __shfl_sync(0xffffffffu, digit, src);
+              above = __shfl_sync(0xffffffffu, above, src);
+              need -= above;
+              pre |= (unsigned long long)digit << shift;
+              pmask |= 255ull << shift;
+              __syncwarp();
+            }
+            if (found) k = pre;
+          }
+          if (!found) {
+            // largest value whose mass still reaches tau; it lies between
+            // the smallest and largest key, so the bits they share are fixed
+            k = 0;
+            for (int bit = common_prefix(key, f0, lane, &k); bit >= 0; --bit) {
+              const unsigned long long cand = k | (1ull << bit);
+              if (mass_ge(cand) >= tau) k = cand;
+            }
           }
           kcut = k;
           // blocks above the cut fall short of tau; add the tied ones in J order

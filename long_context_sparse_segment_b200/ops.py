@@ -250,6 +250,33 @@ def pbs_attention(q, k, v, block, segment, mode="threshold", param=0.9, scale=0.
     return o
 
 
+class PathGraph:
+    """One step of the whole path (``pbs_attention`` on these q, k, v, with
+    the same options) captured once as a CUDA graph. ``replay()`` launches
+    every kernel of the step again as one graph launch on the current
+    stream, on whatever q, k, v hold at that time (copy new inputs into
+    them), and returns the same output tensor (or dict with ``keep``).
+    Buffers, tensor maps and launch shapes are fixed at capture, so nothing
+    is allocated or encoded per replay; inputs must keep their shapes and
+    storage. A first call outside the capture sets the kernels' attributes."""
+
+    def __init__(self, q, k, v, block, segment, mode="threshold", param=0.9, scale=0.0, **kw):
+        dev = q.device
+        call = lambda: pbs_attention(q, k, v, block, segment, mode, param, scale, **kw)
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            call()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.out = call()
+
+    def replay(self):
+        self.graph.replay()
+        return self.out
+
+
 _COPY_STREAMS = {}
 
 

@@ -85,3 +85,46 @@ def test_bench_block_option(dev):
     assert d["config"]["workload"] == "llama8k_b64" and d["config"]["block"] == 64
     assert d["config"]["segment"] == WORKLOADS["llama8k"].segment
     assert d["value"] > 0 and d["roofline"]["achieved"] > 0
+
+
+@pytest.mark.parametrize("queries", ["natural", "fused", "separate"])
+@pytest.mark.parametrize("gather_kv", [False, True])
+def test_graph_of_the_timed_step_computes_the_path(queries, gather_kv, dev):
+    """The step captured as a CUDA graph the way `bench.py --graph` does
+    (events around each step inside the graph) gives the path's output when
+    replayed, also after new inputs are copied into the layer's tensors."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    w = Workload("bench2k", 1, 8, 2, 2048, 128, 128, 512, "topk_frac", 0.3, "per_segment",
+                 0.02)
+    layer = bench.Layer(w, dev, 0, seed_offset=0, gather_kv=gather_kv, queries=queries)
+    bench.run_layer(layer)  # the warm-up step: output buffers, kernel attributes
+    names = ("score", "permute", "select", "attn", "unpermute")
+    ev = {n: (torch.cuda.Event(enable_timing=True, external=True),
+              torch.cuda.Event(enable_timing=True, external=True)) for n in names}
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        o, _ = bench.run_layer(layer, ev)
+    fresh = bench.Layer(w, dev, 1, seed_offset=0)
+    for turn in range(2):
+        if turn:
+            for t, src in ((layer.q, fresh.q), (layer.k, fresh.k), (layer.v, fresh.v)):
+                t.copy_(src)
+        g.replay()
+        ref = pbs.pbs_attention(layer.q, layer.k, layer.v, w.block, w.segment, w.mode, w.param,
+                                permute_q=queries != "natural", gather_kv=gather_kv)
+        torch.cuda.synchronize()
+        assert pbs.device_status() == 0
+        assert torch.equal(o, ref), f"replay {turn}"
+        assert ev["attn"][0].elapsed_time(ev["attn"][1]) > 0
+
+
+def test_bench_graph_option(dev):
+    """--graph replays one CUDA graph per layer in the timed region and says
+    so in its config; its per-step breakdown comes from the graph's events."""
+    d = run_bench("--config", "tiny", "--graph", "--steps", "20", "--warmup", "3",
+                  "--no-cpu-baseline", "--e2e-steps", "1")
+    assert d["config"]["launch"] == "one CUDA graph per layer, replayed"
+    assert d["value"] > 0 and d["breakdown_ms"]["attn"] > 0
+    assert d["breakdown_ms"]["attn"] <= d["ms_per_step"]
