@@ -595,13 +595,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         kp4 = reinterpret_cast<const int4 *>(sKP + vsl * kBN);
       }
+      // Columns past lim_b of block b are hidden: none when the row's list
+      // keeps the block off its own segment (the common step), all when it
+      // does not keep it, the causal limit on the own segment; with carried
+      // positions the own segment's blocks are masked per column instead.
+      const int lim0 = !mine0 ? -1 : (diag0 && !kp4) ? qp - J[0] * kSB : kSB;
+      const int lim1 = !mine1 ? -1 : (diag1 && !kp4) ? qp - J[1] * kSB : kSB;
+      if (lim0 < kSB - 1 || lim1 < kSB - 1) {
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        const bool mine = b ? mine1 : mine0, diag = b ? diag1 : diag0;
-        if (!mine) {
+        for (int c = 0; c < kSB; ++c) {
+          if (c > lim0) v[c] = 0xff800000u;  // -inf
+          if (c > lim1) v[kSB + c] = 0xff800000u;
+        }
+      }
+      if (kp4) {
 #pragma unroll
-          for (int c = 0; c < kSB; ++c) v[b * kSB + c] = 0xff800000u;  // -inf
-        } else if (diag && kp4) {
+        for (int b = 0; b < 2; ++b) {
+          if (!(b ? diag1 : diag0)) continue;
 #pragma unroll
           for (int c4 = 0; c4 < kSB / 4; ++c4) {
             const int4 p = kp4[b * (kSB / 4) + c4];
@@ -611,11 +621,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.z > qp) v[c + 2] = 0xff800000u;
             if (p.w > qp) v[c + 3] = 0xff800000u;
           }
-        } else if (diag) {
-          const int lim = qp - J[b] * kSB;  // last visible column of the block
-#pragma unroll
-          for (int c = 0; c < kSB; ++c)
-            if (c > lim) v[b * kSB + c] = 0xff800000u;
         }
       }
       // row max: eight independent chains over the 128 columns
