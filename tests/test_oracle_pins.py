@@ -270,6 +270,23 @@ def test_block_score_is_mean_of_token_logits():
             assert abs(sigma * qb[0, 0, i] @ kb[0, 0, j] - want) < 1e-13
 
 
+def test_block_scores_map_query_heads_to_their_kv_heads():
+    """block_scores[b, g, I, J] is the mean of the B x B token logits of
+    query head g against KV head g // G (grouped-query attention: G
+    consecutive query heads share one KV head), for every pair, batch and
+    head."""
+    q, k, _ = rand_qkv(17, hq=6, hkv=3, n=32, d=8, b=2)
+    B, G = 8, 2
+    sigma = orc.resolve_scale(None, 8)
+    a = orc.block_scores(orc.block_means(q, B), orc.block_means(k, B), None, G)
+    assert a.shape == (2, 6, 4, 4)
+    for bi in range(2):
+        for g in range(6):
+            tok = sigma * q[bi, g] @ k[bi, g // G].T
+            want = tok.reshape(4, B, 4, B).mean(axis=(1, 3))
+            np.testing.assert_allclose(a[bi, g], want, rtol=0, atol=1e-13)
+
+
 @pytest.mark.parametrize("tau", [0.3, 0.6, 0.9, 0.97])
 def test_threshold_selection_brute_force(tau):
     """Among all subsets T of earlier-segment blocks whose mass with the own
