@@ -131,6 +131,71 @@ def test_identity_permutation_is_plain_block_sparse():
         np.testing.assert_allclose(o[:, g:g + 1], ref, atol=1e-12)
 
 
+def test_attend_blocks_is_masked_library_attention_on_the_permuted_sequence():
+    """attend_blocks on a within-segment key order and grouped heads: each
+    requested query block's rows equal the library routine on the permuted
+    K, V with the token mask 'key block kept and original key position <=
+    query position', query head g reading KV head g // G."""
+    rng = np.random.default_rng(23)
+    q, k, v = rand_qkv(23, b=2, hq=4, hkv=2, n=64, d=8)
+    block, segment = 8, 32
+    kpos = within_segment_perm(rng, 2, 2, 64, segment)
+    kp = orc.gather_rows(k, kpos)
+    vp = orc.gather_rows(v, kpos)
+    idx, cnt, _ = orc.select_blocks(orc.block_means(q, block), orc.block_means(kp, block),
+                                    segment // block, "threshold", 0.7, None, 2)
+    want_blocks = [(0, 0, 7), (0, 3, 2), (1, 1, 4), (1, 2, 0), (1, 3, 5)]
+    got = orc.attend_blocks(q, kp, vp, kpos, None, idx, cnt, block, want_blocks)
+    for t, (bi, g, blk) in enumerate(want_blocks):
+        h = g // 2
+        blockmask = np.zeros((8, 8), dtype=bool)
+        for i in range(8):
+            blockmask[i, idx[bi, g, i, :cnt[bi, g, i]]] = True
+        mask = np.kron(blockmask, np.ones((block, block), dtype=bool)) & \
+            (kpos[bi, h][None, :] <= np.arange(64)[:, None])
+        ref = sdpa(q[bi:bi + 1, g:g + 1], kp[bi:bi + 1, h:h + 1], vp[bi:bi + 1, h:h + 1],
+                   mask=mask)[0, 0]
+        np.testing.assert_allclose(got[t], ref[blk * block:(blk + 1) * block], atol=1e-12)
+
+
+def test_block_flops_counts_the_multiply_adds_of_a_block_loop():
+    """block_flops is twice the multiply-adds that a block-by-block forward
+    performs: a plain loop over the kept blocks that counts every product it
+    forms (q.k per logit, p*v per output element), and whose output matches
+    attend, so that the count is of real work."""
+    q, k, v = rand_qkv(29, hq=2, hkv=1, n=32, d=4)
+    block, segment = 8, 16
+    idx, cnt, _ = orc.select_blocks(orc.block_means(q, block), orc.block_means(k, block),
+                                    segment // block, "topk_frac", 0.5, None, 2)
+    sigma = orc.resolve_scale(None, 4)
+    macs = 0
+    out = np.zeros((1, 2, 32, 4))
+    for g in range(2):
+        for I in range(4):
+            rows = range(I * block, (I + 1) * block)
+            kept = idx[0, g, I, :cnt[0, g, I]]
+            logits = np.full((block, 32), -np.inf)
+            for J in kept:
+                for r in rows:
+                    for c in range(J * block, (J + 1) * block):
+                        acc = 0.0
+                        for e in range(4):
+                            acc += q[0, g, r, e] * k[0, 0, c, e]
+                            macs += 1
+                        if c <= r:
+                            logits[r - I * block, c] = sigma * acc
+            w = np.exp(logits - logits.max(axis=1, keepdims=True))
+            w /= w.sum(axis=1, keepdims=True)
+            for J in kept:
+                for r in rows:
+                    for c in range(J * block, (J + 1) * block):
+                        for e in range(4):
+                            out[0, g, r, e] += w[r - I * block, c] * v[0, 0, c, e]
+                            macs += 1
+    np.testing.assert_allclose(out, orc.attend(q, k, v, None, None, idx, cnt, block), atol=1e-12)
+    assert orc.block_flops(cnt, block, 4) == 2 * macs
+
+
 def test_single_segment_is_dense_causal():
     """S = N: every block is in the on-diagonal segment, so the whole path
     (with its permutation) reproduces dense causal attention."""
