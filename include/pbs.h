@@ -37,6 +37,14 @@
  *   launch nothing. Errors found by a kernel (a wait that ran out, an index
  *   out of range) are recorded in a per-device error word that
  *   pbs_get_device_status reads. Nothing throws across this ABI.
+ * - The calls of the device path (pbs_score, pbs_permute,
+ *   pbs_select_blocks, pbs_attn_fwd and its _unpermute and _gather forms,
+ *   pbs_unpermute) only enqueue work on the given stream: they neither
+ *   synchronise nor allocate, so a sequence of them can be captured into a
+ *   CUDA graph (stream capture) and replayed on whatever the captured
+ *   buffers hold at replay time; shapes, pointers and the softmax scale are
+ *   fixed at capture. The whole path captured that way replays bit for bit
+ *   like the calls themselves.
  */
 #ifndef PBS_H
 #define PBS_H
