@@ -599,6 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // keeps the block off its own segment (the common step), all when it
       // does not keep it, the causal limit on the own segment; with carried
       // positions the own segment's blocks are masked per column instead.
+      // One branch skips the selects when no column is hidden (run on every
+      // step they took ~10 % of the kernel at llama32k).
       const int lim0 = !mine0 ? -1 : (diag0 && !kp4) ? qp - J[0] * kSB : kSB;
       const int lim1 = !mine1 ? -1 : (diag1 && !kp4) ? qp - J[1] * kSB : kSB;
       if (lim0 < kSB - 1 || lim1 < kSB - 1) {
